@@ -1,0 +1,8 @@
+"""Seeded synthetic inputs shared by the tests, the benchmark and the oracle checks.
+
+This package generates operator INPUTS only (geometry, edge features, node
+features, weights, output cotangents). It holds none of the convolution's
+arithmetic, imports neither the CUDA path nor the oracle, and is the one module
+both sides see.
+"""
+from .workloads import CONFIGS, Workload, make_workload  # noqa: F401

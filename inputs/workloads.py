@@ -1,0 +1,209 @@
+"""The five synthetic workloads of the tensor-product convolution.
+
+They stand in for the pages' datasets (LunaTP §5 / App. A sample OMat24 and
+MPTrj structures with periodic neighbour lists; Sobek §5.1 builds radius graphs
+on synthetic positions), none of which is available here.
+
+Recipe (seed = workload id; draw order positions, x, A, grad_out):
+* positions uniform in a cube; workload 1 is an open 6 A box with a 3 A cutoff;
+  workloads 2, 4, 5 are periodic cubes of side (N / rho)^(1/3) with
+  rho = d / (4/3 pi r_c^3), r_c = 5 A, d the target mean degree; workload 3
+  reuses workload 1's positions;
+* edges: every ordered pair i != j closer than r_c (minimum image when periodic),
+  emitted in (src, dst) lexicographic order, so the receiver CSR is a real
+  reordering;
+* Y: component-normalised real spherical harmonics of r_hat_ij, r_ij = r_j - r_i
+  (j sender, i receiver), blocks l = 0..L, m = -l..l, l = 1 ordered (y, z, x);
+* phi: K Bessel functions sqrt(2/r_c) sin(n pi r / r_c) / r times the cosine
+  cutoff (cos(pi r / r_c) + 1) / 2;
+* x, grad_out ~ N(0, 1); A ~ N(0, s) with s the standard deviation
+  1/sqrt(8) (workload 1), 1/sqrt(K) (2-4), 1/sqrt(16*32) (5);
+* floating inputs are drawn in fp64 and rounded once to the workload dtype.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import Optional
+
+import numpy as np
+from scipy.spatial import cKDTree
+from scipy.special import sph_harm_y
+
+
+@dataclass(frozen=True)
+class Config:
+    id: int
+    name: str
+    irreps_in: str
+    sh_lmax: int
+    irreps_out: str
+    K: int
+    mode: str
+    dtype: str          # "f32" | "f64"
+    n_nodes: int
+    box: float          # cube side (A)
+    periodic: bool
+    r_cut: float
+    a_std: float
+    backward: bool
+    positions_from: int = 0   # reuse another workload's positions
+
+
+def _lp(mul: int, lmax: int, all_parities: bool, skip=()) -> str:
+    terms = []
+    for l in range(lmax + 1):
+        nat = "e" if l % 2 == 0 else "o"
+        terms.append(f"{mul}x{l}{nat}")
+        if all_parities and l > 0:
+            terms.append(f"{mul}x{l}{'o' if nat == 'e' else 'e'}")
+    return "+".join(t for t in terms if t not in skip)
+
+
+def _box(n: int, degree: float, r_cut: float) -> float:
+    rho = degree / (4.0 / 3.0 * np.pi * r_cut ** 3)
+    return float((n / rho) ** (1.0 / 3.0))
+
+
+CONFIGS = {
+    1: Config(1, "tiny check f64 uvu (64 nodes, 6 A open box, r_c 3 A)",
+              "8x0e+8x1o+8x2e", 2, _lp(8, 2, True), 8, "uvu", "f64",
+              64, 6.0, False, 3.0, 1.0 / np.sqrt(8.0), True),
+    2: Config(2, "MACE-like channelwise f32 uvu (4096 atoms, ~32 nbrs, 128 ch, L_sh 3)",
+              "128x0e+128x1o", 3, "128x0e+128x1o+128x2e+128x3o", 8, "uvu", "f32",
+              4096, _box(4096, 32.0, 5.0), True, 5.0, 1.0 / np.sqrt(8.0), False),
+    3: Config(3, "tiny geometry f64 uvu, 64 channels, l <= 3",
+              "64x0e+64x1o+64x2e+64x3o", 3, _lp(64, 3, True), 8, "uvu", "f64",
+              64, 6.0, False, 3.0, 1.0 / np.sqrt(8.0), True, positions_from=1),
+    4: Config(4, "large graph f32 uvu (100k atoms, ~40 nbrs, 64 ch, l <= 2)",
+              "64x0e+64x1o+64x2e", 2, _lp(64, 2, True), 8, "uvu", "f32",
+              100_000, _box(100_000, 40.0, 5.0), True, 5.0, 1.0 / np.sqrt(8.0), True),
+    5: Config(5, "fully connected f32 uvw (16384 atoms, ~32 nbrs, 32 ch, l <= 4, K 16)",
+              "32x0e+32x1o+32x2e+32x3o+32x4e", 4, _lp(32, 4, True), 16, "uvw", "f32",
+              16_384, _box(16_384, 32.0, 5.0), True, 5.0, 1.0 / np.sqrt(16.0 * 32.0), True),
+}
+
+
+def _positions(cfg: Config, rng: np.random.Generator) -> np.ndarray:
+    return rng.uniform(0.0, cfg.box, size=(cfg.n_nodes, 3))
+
+
+def radius_graph(pos: np.ndarray, box: float, periodic: bool, r_cut: float):
+    """All ordered pairs (src, dst), src != dst, |r_dst - r_src| < r_cut (min. image)."""
+    if periodic:
+        tree = cKDTree(np.mod(pos, box), boxsize=box)
+    else:
+        tree = cKDTree(pos)
+    pairs = tree.query_pairs(r_cut, output_type="ndarray")
+    if len(pairs) == 0:
+        return np.zeros(0, np.int64), np.zeros(0, np.int64)
+    a = np.concatenate([pairs[:, 0], pairs[:, 1]]).astype(np.int64)
+    b = np.concatenate([pairs[:, 1], pairs[:, 0]]).astype(np.int64)
+    order = np.lexsort((b, a))
+    return a[order], b[order]
+
+
+def edge_vectors(pos, src, dst, box, periodic):
+    """r_ij = r_j - r_i for edge j -> i, i.e. sender minus receiver (minimum image)."""
+    d = pos[src] - pos[dst]
+    if periodic:
+        d = d - box * np.round(d / box)
+    return d
+
+
+def spherical_harmonics(lmax: int, vec: np.ndarray) -> np.ndarray:
+    """Component-normalised real SH, blocks l = 0..lmax, from scipy's complex Y."""
+    v = np.asarray(vec, np.float64)
+    r = np.linalg.norm(v, axis=1)
+    theta = np.arccos(np.clip(v[:, 2] / r, -1.0, 1.0))
+    azim = np.arctan2(v[:, 1], v[:, 0])
+    cols = []
+    for l in range(lmax + 1):
+        s = np.sqrt(4.0 * np.pi)
+        blk = np.zeros((len(v), 2 * l + 1))
+        for m in range(-l, l + 1):
+            if m == 0:
+                blk[:, l] = s * sph_harm_y(l, 0, theta, azim).real
+            elif m > 0:
+                blk[:, l + m] = s * np.sqrt(2.0) * (-1) ** m * sph_harm_y(l, m, theta, azim).real
+            else:
+                blk[:, l + m] = s * np.sqrt(2.0) * (-1) ** (-m) * sph_harm_y(l, -m, theta, azim).imag
+        cols.append(blk)
+    return np.concatenate(cols, axis=1)
+
+
+def bessel_cutoff(r: np.ndarray, K: int, r_cut: float) -> np.ndarray:
+    n = np.arange(1, K + 1, dtype=np.float64)
+    rr = r[:, None]
+    b = np.sqrt(2.0 / r_cut) * np.sin(n[None, :] * np.pi * rr / r_cut) / rr
+    env = 0.5 * (np.cos(np.pi * r / r_cut) + 1.0)
+    return b * env[:, None]
+
+
+def _irreps_dim(s: str) -> int:
+    tot = 0
+    for t in s.split("+"):
+        mul, ir = t.split("x")
+        tot += int(mul) * (2 * int(ir[:-1]) + 1)
+    return tot
+
+
+@dataclass
+class Workload:
+    cfg: Config
+    pos: np.ndarray
+    src: np.ndarray      # COO, int64
+    dst: np.ndarray
+    Y: np.ndarray        # [E, (L+1)^2] in COO order, workload dtype
+    phi: np.ndarray      # [E, K] in COO order, workload dtype
+    x: np.ndarray        # [N, C_x] ir_mul, workload dtype
+    A: np.ndarray        # [K, N_w], workload dtype
+    grad_out: np.ndarray  # [N, C_out], workload dtype
+    n_w: int = field(default=0)
+
+    @property
+    def n_nodes(self) -> int:
+        return self.cfg.n_nodes
+
+    @property
+    def n_edges(self) -> int:
+        return len(self.src)
+
+    @property
+    def np_dtype(self):
+        return np.float32 if self.cfg.dtype == "f32" else np.float64
+
+
+def make_workload(cfg_id: int, n_w: int, n_nodes: Optional[int] = None,
+                  edge_keep: Optional[float] = None) -> Workload:
+    """Build workload ``cfg_id``.
+
+    n_w (the weight count of the operator's path layout) is an argument so that
+    this module stays free of the operator's path rules. ``n_nodes`` shrinks a
+    periodic workload at fixed density (for fast tests); ``edge_keep`` keeps a
+    seeded fraction of the edges (for workspace-versus-edge-count checks).
+    """
+    cfg = CONFIGS[cfg_id]
+    if n_nodes is not None and n_nodes != cfg.n_nodes:
+        if not cfg.periodic:
+            raise ValueError("only periodic workloads can be resized")
+        deg = cfg.n_nodes / cfg.box ** 3
+        cfg = Config(**{**cfg.__dict__, "n_nodes": n_nodes,
+                        "box": float((n_nodes / deg) ** (1.0 / 3.0))})
+    rng = np.random.default_rng(cfg.id)
+    if cfg.positions_from:
+        pos = _positions(CONFIGS[cfg.positions_from], np.random.default_rng(cfg.positions_from))
+    else:
+        pos = _positions(cfg, rng)
+    src, dst = radius_graph(pos, cfg.box, cfg.periodic, cfg.r_cut)
+    if edge_keep is not None:
+        keep = np.random.default_rng(1000 + cfg.id).random(len(src)) < edge_keep
+        src, dst = src[keep], dst[keep]
+    vec = edge_vectors(pos, src, dst, cfg.box, cfg.periodic)
+    r = np.linalg.norm(vec, axis=1)
+    dt = np.float32 if cfg.dtype == "f32" else np.float64
+    Y = spherical_harmonics(cfg.sh_lmax, vec).astype(dt)
+    phi = bessel_cutoff(r, cfg.K, cfg.r_cut).astype(dt)
+    x = rng.normal(size=(cfg.n_nodes, _irreps_dim(cfg.irreps_in))).astype(dt)
+    A = (rng.normal(size=(cfg.K, n_w)) * cfg.a_std).astype(dt)
+    g = rng.normal(size=(cfg.n_nodes, _irreps_dim(cfg.irreps_out))).astype(dt)
+    return Workload(cfg, pos, src, dst, Y, phi, x, A, g, n_w)

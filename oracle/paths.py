@@ -1,0 +1,128 @@
+"""Path enumeration and weight layout (oracle; test infrastructure).
+
+Sobek §2.2: an input irrep (l_in, s_in) couples with a spherical-harmonic irrep
+(l_sh, s_sh) into l_out in |l_in - l_sh| .. l_in + l_sh with parity s_in * s_sh.
+LunaTP §2.1 calls each coupling (l1, l2) -> l a path. Sobek §2.4: path pi carries
+n_pi = C_in C_out weights for fully connected (uvw) mixing and n_pi = C for
+channelwise (uvu) mixing; N_w = sum_pi n_pi.
+
+Reading of the enumeration order (the pages are silent; it fixes the layout of A
+and of the output sums): for each input block in the order written, for l2 =
+0..L_sh ascending, for l3 = |l1-l2|..l1+l2 ascending, one path to every output
+block of degree l3 and parity p1*p2 (in output order). Output blocks receive the
+sum over all their paths. Spherical harmonics carry their natural parity
+(-1)^l2 unless an explicit list of (l2, p2) is given.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import List, Sequence, Tuple, Union
+
+from . import irreps as _ir
+from .cg import real_cg_sparse
+
+
+@dataclass(frozen=True)
+class Path:
+    index: int
+    i_in: int       # input block
+    l1: int
+    p1: int
+    l2: int
+    p2: int
+    l3: int
+    p3: int
+    i_out: int      # output block
+    mul_in: int
+    mul_out: int
+    w_off: int      # first column of this path in A [K, N_w]
+    n_w: int        # columns of this path
+
+
+def sh_irreps(sh: Union[int, Sequence[Tuple[int, int]]]) -> List[Tuple[int, int]]:
+    if isinstance(sh, int):
+        return [(l, (-1) ** l) for l in range(sh + 1)]
+    return [(int(l), int(p)) for l, p in sh]
+
+
+def y_offset(l2: int) -> int:
+    """Blocks of Y are l = 0..L in order, so block l starts at l^2."""
+    return l2 * l2
+
+
+def enumerate_paths(irreps_in: str, sh, irreps_out: str, mode: str) -> List[Path]:
+    bin_ = _ir.parse(irreps_in)
+    bout = _ir.parse(irreps_out)
+    shl = sh_irreps(sh)
+    paths: List[Path] = []
+    w = 0
+    for i1, b1 in enumerate(bin_):
+        for (l2, p2) in shl:
+            for l3 in range(abs(b1.l - l2), b1.l + l2 + 1):
+                p3 = b1.p * p2
+                for io, bo in enumerate(bout):
+                    if bo.l != l3 or bo.p != p3:
+                        continue
+                    if mode == "uvu":
+                        if bo.mul != b1.mul:
+                            raise ValueError("uvu needs equal input and output multiplicity "
+                                             f"on every path, got {b1.mul} -> {bo.mul}")
+                        nw = b1.mul
+                    elif mode == "uvw":
+                        nw = b1.mul * bo.mul
+                    else:
+                        raise ValueError(mode)
+                    paths.append(Path(len(paths), i1, b1.l, b1.p, l2, p2, l3, p3, io,
+                                      b1.mul, bo.mul, w, nw))
+                    w += nw
+    return paths
+
+
+def n_weights(paths: List[Path]) -> int:
+    return sum(p.n_w for p in paths)
+
+
+def concatenated_out_mul(irreps_in: str, sh, out_lp: Sequence[Tuple[int, int]]):
+    """Per-path concatenated uvu output multiplicity per output (l, p).
+
+    LunaTP Table 1 lists, for each case, output irreps whose multiplicity is the
+    sum over paths into (l, p) of the path's input multiplicity (uvu, one output
+    slot per path). Used as a pin of the enumeration rule.
+    """
+    bin_ = _ir.parse(irreps_in)
+    shl = sh_irreps(sh)
+    want = set((int(l), int(p)) for l, p in out_lp)
+    tot = {lp: 0 for lp in want}
+    for b1 in bin_:
+        for (l2, p2) in shl:
+            for l3 in range(abs(b1.l - l2), b1.l + l2 + 1):
+                key = (l3, b1.p * p2)
+                if key in want:
+                    tot[key] += b1.mul
+    return tot
+
+
+def work_model(paths: List[Path], n_nodes: int, n_edges: int, K: int, mode: str) -> dict:
+    """Algorithmic flop counts (FMA = 2 flops) of the streamed schedule.
+
+    uvu (Sobek §3.1 order, w live only until consumed): per edge, channel, path:
+      K (w = phi . A) + nnz (CG contraction) + (2 l3 + 1) (weighted accumulate).
+    uvw (Sobek §4.2, Eqs. 32-35): per edge, path: 2 C_in nnz (Eq. 32) +
+      2 K C_in (2 l3 + 1) (Eq. 33); per receiver, path: 2 (2 l3 + 1) K C_in C_out
+      (Eq. 34-35).
+    """
+    fwd = 0
+    bwd = 0
+    for p in paths:
+        nnz = len(real_cg_sparse(p.l1, p.l2, p.l3))
+        d3 = 2 * p.l3 + 1
+        if mode == "uvu":
+            C = p.mul_in
+            fwd += 2 * n_edges * C * (K + nnz + d3)
+            bwd += 2 * n_edges * C * (3 * K + 3 * nnz + 2 * d3)
+        else:
+            e = n_edges * (2 * p.mul_in * nnz + 2 * K * p.mul_in * d3)
+            r = n_nodes * 2 * d3 * K * p.mul_in * p.mul_out
+            fwd += e + r
+            bwd += r + e + n_edges * (4 * K * p.mul_in * d3 + 4 * p.mul_in * nnz)
+    return {"fwd_flops": fwd, "bwd_flops": bwd}
