@@ -1,0 +1,345 @@
+// C ABI of the tensor-product convolution library (declarations in tpconv.h).
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "cg_host.h"
+#include "kernels.h"
+#include "plan.h"
+#include "tpconv.h"
+
+struct tp_plan_s {
+  tpc::Plan p;
+};
+
+namespace tpc {
+namespace {
+
+thread_local std::string g_msg;
+
+int fail(int status, const std::string& m) {
+  g_msg = m;
+  return status;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  return fail(TP_ECUDA, std::string(where) + ": " + cudaGetErrorString(e));
+}
+
+// Per-device error word: kernels set bits here instead of trapping.
+__device__ int g_error_word;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_err_mu;
+int* g_err_ptr[kMaxDevices] = {};
+
+int error_word(int** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(TP_EUNSUPPORTED, "device ordinal above 63");
+  std::lock_guard<std::mutex> lk(g_err_mu);
+  if (!g_err_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_error_word);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+    g_err_ptr[dev] = static_cast<int*>(ptr);
+  }
+  *out = g_err_ptr[dev];
+  return TP_OK;
+}
+
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_sizes(long long N, long long E) {
+  if (N < 0 || E < 0) return fail(TP_EINVAL, "negative node or edge count");
+  if (N >= (1LL << 31) - 1 || E >= (1LL << 31) - 1) return fail(TP_EINVAL, "N and E must be below 2^31 - 1");
+  return TP_OK;
+}
+
+template <typename P>
+void copy_tables(P& prm, const std::vector<TileD>& tiles, const std::vector<PathD>& paths) {
+  std::memset(prm.tiles, 0, sizeof(prm.tiles));
+  std::memset(prm.paths, 0, sizeof(prm.paths));
+  std::memcpy(prm.tiles, tiles.data(), tiles.size() * sizeof(TileD));
+  std::memcpy(prm.paths, paths.data(), paths.size() * sizeof(PathD));
+  prm.n_tiles = (int)tiles.size();
+}
+
+template <typename T, template <typename, int, int> class L, typename Prm>
+cudaError_t dispatch_kc(const Plan& P, const Prm& prm, cudaStream_t s) {
+  if (P.KP == 8 && P.CPL == 1) return L<T, 8, 1>::run(prm, s);
+  if (P.KP == 16 && P.CPL == 1) return L<T, 16, 1>::run(prm, s);
+  if constexpr (std::is_same<T, float>::value) {
+    if (P.KP == 8 && P.CPL == 2) return L<T, 8, 2>::run(prm, s);
+    if (P.KP == 16 && P.CPL == 2) return L<T, 16, 2>::run(prm, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <typename T, int KP, int CPL>
+struct FwdL {
+  static cudaError_t run(const UvuFwdParams<T>& p, cudaStream_t s) { return launch_uvu_fwd<T, KP, CPL>(p, s); }
+};
+template <typename T, int KP, int CPL>
+struct EdgeL {
+  static cudaError_t run(const UvuEdgeParams<T>& p, cudaStream_t s) { return launch_uvu_edge<T, KP, CPL>(p, s); }
+};
+template <typename T, int KP, int CPL>
+struct SrcL {
+  static cudaError_t run(const UvuSrcParams<T>& p, cudaStream_t s) { return launch_uvu_src<T, KP, CPL>(p, s); }
+};
+
+template <typename T>
+int forward_uvu(const Plan& P, const void* x, const void* Y, const void* phi, const void* A,
+                const int* rowptr, const int* senders, int N, int E, void* out, int* err, cudaStream_t s) {
+  UvuFwdParams<T> prm;
+  prm.x = (const T*)x; prm.Y = (const T*)Y; prm.phi = (const T*)phi; prm.A = (const T*)A;
+  prm.rowptr = rowptr; prm.senders = senders; prm.out = (T*)out; prm.err = err;
+  prm.N = N; prm.E = E; prm.K = P.K; prm.c_in = P.c_in; prm.c_out = P.c_out; prm.dim_y = P.dim_y;
+  prm.n_w = (int)P.n_w;
+  copy_tables(prm, P.out_tiles, P.paths_by_out);
+  cudaError_t e = dispatch_kc<T, FwdL>(P, prm, s);
+  return e == cudaSuccess ? TP_OK : cuda_fail(e, "uvu forward launch");
+}
+
+template <typename T>
+int backward_uvu(const Plan& P, const void* x, const void* Y, const void* phi, const void* A,
+                 const int* rowptr, const int* senders, const int* colptr, const int* srcedge,
+                 const int* srcrecv, const void* gout, int N, int E, void* gx, void* gY, void* gphi,
+                 void* gA, void* ws, int* err, cudaStream_t s) {
+  UvuEdgeParams<T> ep;
+  ep.x = (const T*)x; ep.Y = (const T*)Y; ep.phi = (const T*)phi; ep.A = (const T*)A;
+  ep.gout = (const T*)gout; ep.rowptr = rowptr; ep.senders = senders;
+  ep.gY = (T*)gY; ep.gphi = (T*)gphi; ep.err = err;
+  ep.N = N; ep.E = E; ep.K = P.K; ep.c_in = P.c_in; ep.c_out = P.c_out; ep.dim_y = P.dim_y;
+  ep.n_w = (int)P.n_w; ep.n_paths = (int)P.paths_canon.size();
+  std::memset(ep.paths, 0, sizeof(ep.paths));
+  std::memcpy(ep.paths, P.paths_canon.data(), P.paths_canon.size() * sizeof(PathD));
+  cudaError_t e = dispatch_kc<T, EdgeL>(P, ep, s);
+  if (e != cudaSuccess) return cuda_fail(e, "uvu edge pass launch");
+
+  UvuSrcParams<T> sp;
+  sp.x = (const T*)x; sp.Y = (const T*)Y; sp.phi = (const T*)phi; sp.A = (const T*)A;
+  sp.gout = (const T*)gout; sp.colptr = colptr; sp.srcedge = srcedge; sp.srcrecv = srcrecv;
+  sp.gx = (T*)gx; sp.apart = (T*)ws; sp.err = err;
+  sp.N = N; sp.E = E; sp.K = P.K; sp.c_in = P.c_in; sp.c_out = P.c_out; sp.dim_y = P.dim_y;
+  sp.n_w = (int)P.n_w;
+  sp.n_slots = uvu_src_slots(P, N);
+  copy_tables(sp, P.in_tiles, P.paths_by_in);
+  e = dispatch_kc<T, SrcL>(P, sp, s);
+  if (e != cudaSuccess) return cuda_fail(e, "uvu source pass launch");
+  e = launch_reduce_slots<T>((const T*)ws, (T*)gA, sp.n_slots, (long long)P.K * P.n_w, s);
+  return e == cudaSuccess ? TP_OK : cuda_fail(e, "grad_A reduction launch");
+}
+
+}  // namespace
+}  // namespace tpc
+
+using namespace tpc;
+
+extern "C" {
+
+int tp_conv_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_radial, int mode,
+                 int dtype, tp_plan_t* plan) {
+  if (!plan) return fail(TP_EINVAL, "plan output pointer is NULL");
+  *plan = nullptr;
+  auto* h = new (std::nothrow) tp_plan_s;
+  if (!h) return fail(TP_EINVAL, "out of host memory");
+  std::string msg;
+  const int st = make_plan(irreps_in, sh_lmax, irreps_out, n_radial, mode, dtype, h->p, msg);
+  if (st != TP_OK) {
+    delete h;
+    return fail(st, msg);
+  }
+  *plan = h;
+  return TP_OK;
+}
+
+int tp_conv_plan_destroy(tp_plan_t plan) {
+  delete plan;
+  return TP_OK;
+}
+
+int tp_conv_plan_info(tp_plan_t plan, tp_plan_info_t* info) {
+  if (!plan || !info) return fail(TP_EINVAL, "NULL plan or info");
+  const Plan& P = plan->p;
+  std::memset(info, 0, sizeof(*info));
+  info->c_in = P.c_in; info->c_out = P.c_out; info->dim_y = P.dim_y; info->n_radial = P.K;
+  info->n_paths = (int)P.paths.size(); info->mode = P.mode; info->dtype = P.dtype;
+  info->sh_lmax = P.sh_lmax; info->lmax = P.lmax; info->n_w = P.n_w;
+  return TP_OK;
+}
+
+int tp_conv_plan_path(tp_plan_t plan, int index, tp_path_info_t* info) {
+  if (!plan || !info) return fail(TP_EINVAL, "NULL plan or info");
+  const Plan& P = plan->p;
+  if (index < 0 || index >= (int)P.paths.size()) return fail(TP_EINVAL, "path index out of range");
+  const HostPath& h = P.paths[index];
+  std::memset(info, 0, sizeof(*info));
+  info->l1 = h.l1; info->p1 = h.p1; info->l2 = h.l2; info->p2 = h.p2; info->l3 = h.l3; info->p3 = h.p3;
+  info->block_in = h.i_in; info->block_out = h.i_out; info->mul_in = h.mul_in; info->mul_out = h.mul_out;
+  info->x_off = h.x_off; info->out_off = h.out_off; info->w_off = h.w_off; info->n_w = h.n_w;
+  info->nnz = h.nnz;
+  return TP_OK;
+}
+
+int tp_conv_plan_cg(tp_plan_t plan, int index, int32_t* m1, int32_t* m2, int32_t* m3, double* c,
+                    int capacity) {
+  if (!plan) return fail(TP_EINVAL, "NULL plan");
+  const Plan& P = plan->p;
+  if (index < 0 || index >= (int)P.paths.size()) return fail(TP_EINVAL, "path index out of range");
+  const HostPath& h = P.paths[index];
+  auto e = real_cg_sparse(h.l1, h.l2, h.l3);
+  const int n = (int)e.size();
+  if (capacity > 0 && (!m1 || !m2 || !m3 || !c)) return fail(TP_EINVAL, "NULL output array");
+  for (int k = 0; k < n && k < capacity; ++k) {
+    m1[k] = e[k].m1; m2[k] = e[k].m2; m3[k] = e[k].m3; c[k] = e[k].c;
+  }
+  return n;
+}
+
+int tp_conv_work_model(tp_plan_t plan, int64_t n_nodes, int64_t n_edges, int pass, double* flops,
+                       double* bytes) {
+  if (!plan || !flops || !bytes) return fail(TP_EINVAL, "NULL argument");
+  if (pass != 0 && pass != 1) return fail(TP_EINVAL, "pass must be 0 or 1");
+  work_model(plan->p, n_nodes, n_edges, pass, *flops, *bytes);
+  return TP_OK;
+}
+
+int tp_conv_workspace_size(tp_plan_t plan, int64_t n_nodes, int pass, size_t* bytes) {
+  if (!plan || !bytes) return fail(TP_EINVAL, "NULL argument");
+  if (pass != 0 && pass != 1) return fail(TP_EINVAL, "pass must be 0 or 1");
+  if (n_nodes < 0) return fail(TP_EINVAL, "negative node count");
+  *bytes = workspace_bytes(plan->p, n_nodes, pass);
+  return TP_OK;
+}
+
+int tp_csr_workspace_size(int64_t n_nodes, size_t* bytes) {
+  if (!bytes || n_nodes < 0) return fail(TP_EINVAL, "bad argument");
+  *bytes = csr_workspace_bytes(n_nodes);
+  return TP_OK;
+}
+
+int tp_csr_build(int64_t n_nodes, int64_t n_edges, const int32_t* src, const int32_t* dst,
+                 int32_t* rowptr, int32_t* senders, int32_t* perm, void* ws, size_t ws_bytes,
+                 void* stream) {
+  int st = check_sizes(n_nodes, n_edges);
+  if (st) return st;
+  if (!rowptr || !ws || (n_edges > 0 && (!src || !dst || !senders || !perm)))
+    return fail(TP_EINVAL, "NULL device pointer");
+  if (ws_bytes < csr_workspace_bytes(n_nodes)) return fail(TP_EWORKSPACE, "CSR workspace too small");
+  int* err = nullptr;
+  if ((st = error_word(&err))) return st;
+  cudaError_t e = csr_build((int)n_nodes, (int)n_edges, src, dst, rowptr, senders, perm, ws, err,
+                            (cudaStream_t)stream);
+  return e == cudaSuccess ? TP_OK : cuda_fail(e, "tp_csr_build");
+}
+
+int tp_csr_transpose(int64_t n_nodes, int64_t n_edges, const int32_t* rowptr, const int32_t* senders,
+                     int32_t* colptr, int32_t* srcedge, int32_t* srcrecv, void* ws, size_t ws_bytes,
+                     void* stream) {
+  int st = check_sizes(n_nodes, n_edges);
+  if (st) return st;
+  if (!rowptr || !colptr || !ws || (n_edges > 0 && (!senders || !srcedge || !srcrecv)))
+    return fail(TP_EINVAL, "NULL device pointer");
+  if (ws_bytes < csr_workspace_bytes(n_nodes)) return fail(TP_EWORKSPACE, "CSR workspace too small");
+  int* err = nullptr;
+  if ((st = error_word(&err))) return st;
+  cudaError_t e = csr_transpose((int)n_nodes, (int)n_edges, rowptr, senders, colptr, srcedge, srcrecv,
+                                ws, err, (cudaStream_t)stream);
+  return e == cudaSuccess ? TP_OK : cuda_fail(e, "tp_csr_transpose");
+}
+
+int tp_conv_forward(tp_plan_t plan, const void* x, const void* Y, const void* phi, const void* A,
+                    const int32_t* rowptr, const int32_t* senders, int64_t n_nodes, int64_t n_edges,
+                    void* out, void* ws, size_t ws_bytes, void* stream) {
+  if (!plan) return fail(TP_EINVAL, "NULL plan");
+  const Plan& P = plan->p;
+  int st = check_sizes(n_nodes, n_edges);
+  if (st) return st;
+  if (n_nodes == 0) return TP_OK;
+  if (!x || !A || !rowptr || !out || (n_edges > 0 && (!Y || !phi || !senders)))
+    return fail(TP_EINVAL, "NULL device pointer");
+  if (!al16(x) || !al16(A) || !al16(out) || (n_edges > 0 && (!al16(Y) || !al16(phi))))
+    return fail(TP_EINVAL, "floating-point buffers must be 16-byte aligned");
+  if (ws_bytes < workspace_bytes(P, n_nodes, 0)) return fail(TP_EWORKSPACE, "workspace too small");
+  int* err = nullptr;
+  if ((st = error_word(&err))) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (P.mode != TP_UVU) return fail(TP_EUNSUPPORTED, "uvw forward is not built yet");
+  return P.dtype == TP_F32
+             ? forward_uvu<float>(P, x, Y, phi, A, rowptr, senders, (int)n_nodes, (int)n_edges, out, err, s)
+             : forward_uvu<double>(P, x, Y, phi, A, rowptr, senders, (int)n_nodes, (int)n_edges, out, err, s);
+}
+
+int tp_conv_backward(tp_plan_t plan, const void* x, const void* Y, const void* phi, const void* A,
+                     const int32_t* rowptr, const int32_t* senders, const int32_t* colptr,
+                     const int32_t* srcedge, const int32_t* srcrecv, const void* grad_out,
+                     int64_t n_nodes, int64_t n_edges, void* grad_x, void* grad_Y, void* grad_phi,
+                     void* grad_A, void* ws, size_t ws_bytes, void* stream) {
+  if (!plan) return fail(TP_EINVAL, "NULL plan");
+  const Plan& P = plan->p;
+  int st = check_sizes(n_nodes, n_edges);
+  if (st) return st;
+  if (!x || !A || !rowptr || !colptr || !grad_out || !grad_x || !grad_A ||
+      (n_edges > 0 && (!Y || !phi || !senders || !srcedge || !srcrecv || !grad_Y || !grad_phi)))
+    return fail(TP_EINVAL, "NULL device pointer");
+  const void* f[] = {x, A, grad_out, grad_x, grad_A};
+  for (const void* q : f)
+    if (!al16(q)) return fail(TP_EINVAL, "floating-point buffers must be 16-byte aligned");
+  if (n_edges > 0 && (!al16(Y) || !al16(phi) || !al16(grad_Y) || !al16(grad_phi)))
+    return fail(TP_EINVAL, "floating-point buffers must be 16-byte aligned");
+  if (ws_bytes < workspace_bytes(P, n_nodes, 1) || (!ws && workspace_bytes(P, n_nodes, 1) > 0))
+    return fail(TP_EWORKSPACE, "workspace too small");
+  int* err = nullptr;
+  if ((st = error_word(&err))) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (P.mode != TP_UVU) return fail(TP_EUNSUPPORTED, "uvw backward is not built yet");
+  if (n_nodes == 0) {
+    cudaError_t e = cudaMemsetAsync(grad_A, 0, (size_t)P.K * P.n_w * (P.dtype == TP_F32 ? 4 : 8), s);
+    return e == cudaSuccess ? TP_OK : cuda_fail(e, "memset grad_A");
+  }
+  return P.dtype == TP_F32
+             ? backward_uvu<float>(P, x, Y, phi, A, rowptr, senders, colptr, srcedge, srcrecv, grad_out,
+                                   (int)n_nodes, (int)n_edges, grad_x, grad_Y, grad_phi, grad_A, ws, err, s)
+             : backward_uvu<double>(P, x, Y, phi, A, rowptr, senders, colptr, srcedge, srcrecv, grad_out,
+                                    (int)n_nodes, (int)n_edges, grad_x, grad_Y, grad_phi, grad_A, ws, err, s);
+}
+
+int tp_get_device_error(void* stream) {
+  int* err = nullptr;
+  int st = error_word(&err);
+  if (st) return st;
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int v = 0;
+  e = cudaMemcpy(&v, err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read error word");
+  if (v) {
+    const int zero = 0;
+    e = cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "clear error word");
+  }
+  if (v & kErrIndex) return fail(TP_EDEVICE_INDEX, "a kernel met an index outside its range");
+  if (v & kErrCsr) return fail(TP_EDEVICE_CSR, "a kernel met a bad row pointer");
+  return TP_OK;
+}
+
+const char* tp_status_string(int status) {
+  switch (status) {
+    case TP_OK: return "ok";
+    case TP_EINVAL: return "invalid argument";
+    case TP_EUNSUPPORTED: return "unsupported contract";
+    case TP_ECUDA: return "CUDA runtime error";
+    case TP_EWORKSPACE: return "workspace too small";
+    case TP_EDEVICE_INDEX: return "device: index out of range";
+    case TP_EDEVICE_CSR: return "device: bad row pointer";
+    default: return "unknown status";
+  }
+}
+
+const char* tp_last_error_message(void) { return g_msg.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,236 @@
+// Shared device-side definitions of the tensor-product convolution kernels.
+//
+// Layouts (Sobek §4.5: ir_mul, channels contiguous inside each irrep block):
+//   x   [N, C_x]      row j: blocks in irreps order, each [2l+1][mul]
+//   out [N, C_out]    same layout for the output irreps
+//   Y   [E, (L+1)^2]  CSR edge order, blocks l = 0..L, m = -l..l
+//   phi [E, K]        CSR edge order
+//   A   [K, N_w]      path pi in columns [w_off, w_off + n_w); uvu column = u,
+//                     uvw column = u * C_out + w
+// Indices are int32; scalars are float or double (the plan's dtype).
+#pragma once
+
+#include <cstdint>
+#include <type_traits>
+#include <utility>
+
+#include "cg_table.inc"
+#include "tpconv_limits.h"
+
+namespace tpc {
+
+using cgt::Pair;
+using cgt::Term;
+
+// ------------------------------------------------------------------ descriptors
+
+struct PathD {          // one coupling path (l1, l2) -> l3
+  int8_t l1, l2, l3, pad;
+  int x_off;            // input block offset in an x row
+  int out_off;          // output block offset in an out row
+  int w_off;            // first column of the path in A
+  int mul_in;
+  int mul_out;
+};
+
+struct TileD {          // one channel tile of one irrep block
+  int l;                // degree of the block
+  int off;              // block offset in its row
+  int mul;              // block multiplicity
+  int ch0;              // first channel of the tile
+  int nch;              // channels in the tile
+  int pbeg, pend;       // paths of the block, in the kernel's path array
+};
+
+// Device error word bits (read back by tp_get_device_error).
+enum : int { kErrIndex = 1, kErrCsr = 2 };
+
+template <typename T>
+struct UvuFwdParams {
+  const T* x; const T* Y; const T* phi; const T* A;
+  const int* rowptr; const int* senders;
+  T* out; int* err;
+  int N, E, K, c_in, c_out, dim_y, n_w;
+  int n_tiles;
+  TileD tiles[kMaxTiles];     // one per (output block, channel tile)
+  PathD paths[kMaxPaths];     // grouped by output block
+};
+
+template <typename T>
+struct UvuEdgeParams {        // backward: edge-owned grad_phi, grad_Y
+  const T* x; const T* Y; const T* phi; const T* A; const T* gout;
+  const int* rowptr; const int* senders;
+  T* gY; T* gphi; int* err;
+  int N, E, K, c_in, c_out, dim_y, n_w;
+  int n_paths;
+  PathD paths[kMaxPaths];     // canonical order
+};
+
+template <typename T>
+struct UvuSrcParams {         // backward: source-owned grad_x, grad_A partials
+  const T* x; const T* Y; const T* phi; const T* A; const T* gout;
+  const int* colptr; const int* srcedge; const int* srcrecv;
+  T* gx; T* apart; int* err;
+  int N, E, K, c_in, c_out, dim_y, n_w;
+  int n_tiles, n_slots;
+  TileD tiles[kMaxTiles];     // one per (input block, channel tile)
+  PathD paths[kMaxPaths];     // grouped by input block
+};
+
+// ------------------------------------------------------------------ compile-time helpers
+
+template <typename F, int... I>
+__device__ __forceinline__ void static_for_impl(F&& f, std::integer_sequence<int, I...>) {
+  (f(std::integral_constant<int, I>{}), ...);
+}
+
+template <int N, typename F>
+__device__ __forceinline__ void static_for(F&& f) {
+  static_for_impl(f, std::make_integer_sequence<int, N>{});
+}
+
+__host__ __device__ constexpr bool triangle(int a, int b, int c) {
+  return c >= (a > b ? a - b : b - a) && c <= a + b;
+}
+
+// True if pair P of CG<L1,L2,L3> is the first pair that writes output component m3.
+template <class CGp>
+__host__ __device__ constexpr bool first_m3(int P) {
+  for (int k = 0; k < P; ++k)
+    if (CGp::pair[k].m3 == CGp::pair[P].m3) return false;
+  return true;
+}
+// True if pair P is the first pair that reads input component m1.
+template <class CGp>
+__host__ __device__ constexpr bool first_m1(int P) {
+  for (int k = 0; k < P; ++k)
+    if (CGp::pair[k].m1 == CGp::pair[P].m1) return false;
+  return true;
+}
+// True if component m3 of CG<L1,L2,L3> receives any pair.
+template <class CGp>
+__host__ __device__ constexpr bool has_m3(int m3) {
+  for (int k = 0; k < CGp::npair; ++k)
+    if (CGp::pair[k].m3 == m3) return true;
+  return false;
+}
+template <class CGp>
+__host__ __device__ constexpr bool has_m1(int m1) {
+  for (int k = 0; k < CGp::npair; ++k)
+    if (CGp::pair[k].m1 == m1) return true;
+  return false;
+}
+
+// cY = sum over the terms of pair P of c * y[m2] (y holds the degree-L2 block).
+template <typename T, class CGp, int P>
+__device__ __forceinline__ T pair_coef(const T* y) {
+  constexpr Pair pr = CGp::pair[P];
+  T cy = T(CGp::term[pr.start].c) * y[CGp::term[pr.start].m2];
+  static_for<pr.n - 1>([&](auto t) {
+    constexpr Term tm = CGp::term[pr.start + 1 + decltype(t)::value];
+    cy = fma(T(tm.c), y[tm.m2], cy);
+  });
+  return cy;
+}
+
+// Call f(integral_constant<L1>, integral_constant<L2>) for the runtime (l1, l2)
+// among the pairs that can couple into L3.
+template <int L3, typename F>
+__device__ __forceinline__ void dispatch_l1l2(int l1, int l2, F&& f) {
+  static_for<kLmax + 1>([&](auto A1) {
+    static_for<kLmax + 1>([&](auto A2) {
+      constexpr int a = decltype(A1)::value, b = decltype(A2)::value;
+      if constexpr (triangle(a, b, L3)) {
+        if (l1 == a && l2 == b) f(A1, A2);
+      }
+    });
+  });
+}
+
+// Same for (l2, l3) at fixed L1.
+template <int L1, typename F>
+__device__ __forceinline__ void dispatch_l2l3(int l2, int l3, F&& f) {
+  static_for<kLmax + 1>([&](auto A2) {
+    static_for<kLmax + 1>([&](auto A3) {
+      constexpr int b = decltype(A2)::value, c = decltype(A3)::value;
+      if constexpr (triangle(L1, b, c)) {
+        if (l2 == b && l3 == c) f(A2, A3);
+      }
+    });
+  });
+}
+
+// Same for one degree.
+template <typename F>
+__device__ __forceinline__ void dispatch_l(int l, F&& f) {
+  static_for<kLmax + 1>([&](auto A) {
+    if (l == decltype(A)::value) f(A);
+  });
+}
+
+// ------------------------------------------------------------------ memory helpers
+
+template <typename T>
+__device__ __forceinline__ T ldg(const T* p) { return __ldg(p); }
+
+// Load CPL consecutive scalars (8-byte aligned when CPL*sizeof(T) == 8).
+template <int CPL, typename T>
+__device__ __forceinline__ void load_ch(T (&v)[CPL], const T* p) {
+  if constexpr (CPL == 2 && std::is_same<T, float>::value) {
+    float2 t = __ldg(reinterpret_cast<const float2*>(p));
+    v[0] = t.x; v[1] = t.y;
+  } else if constexpr (CPL == 4 && std::is_same<T, float>::value) {
+    float4 t = __ldg(reinterpret_cast<const float4*>(p));
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+  } else if constexpr (CPL == 2 && std::is_same<T, double>::value) {
+    double2 t = __ldg(reinterpret_cast<const double2*>(p));
+    v[0] = t.x; v[1] = t.y;
+  } else {
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) v[c] = __ldg(p + c);
+  }
+}
+
+template <int CPL, typename T>
+__device__ __forceinline__ void store_ch(T* p, const T (&v)[CPL]) {
+  if constexpr (CPL == 2 && std::is_same<T, float>::value) {
+    *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+  } else if constexpr (CPL == 4 && std::is_same<T, float>::value) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  } else if constexpr (CPL == 2 && std::is_same<T, double>::value) {
+    *reinterpret_cast<double2*>(p) = make_double2(v[0], v[1]);
+  } else {
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) p[c] = v[c];
+  }
+}
+
+// K radial values of one edge, zero-padded to KP.
+template <int KP, typename T>
+__device__ __forceinline__ void load_phi(T (&ph)[KP], const T* row, int K) {
+  if (K == KP) {
+    if constexpr (std::is_same<T, float>::value && KP % 4 == 0) {
+#pragma unroll
+      for (int q = 0; q < KP; q += 4) {
+        float4 t = __ldg(reinterpret_cast<const float4*>(row + q));
+        ph[q] = t.x; ph[q + 1] = t.y; ph[q + 2] = t.z; ph[q + 3] = t.w;
+      }
+      return;
+    } else if constexpr (std::is_same<T, double>::value && KP % 2 == 0) {
+#pragma unroll
+      for (int q = 0; q < KP; q += 2) {
+        double2 t = __ldg(reinterpret_cast<const double2*>(row + q));
+        ph[q] = t.x; ph[q + 1] = t.y;
+      }
+      return;
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < KP; ++q) ph[q] = q < K ? __ldg(row + q) : T(0);
+}
+
+__device__ __forceinline__ void raise_error(int* err, int bit) {
+  if ((threadIdx.x & 31) == 0) atomicOr(err, bit);
+}
+
+}  // namespace tpc

@@ -1,0 +1,35 @@
+// Launchers of the tensor-product convolution kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace tpc {
+
+template <typename T, int KP, int CPL>
+cudaError_t launch_uvu_fwd(const UvuFwdParams<T>& p, cudaStream_t s);
+
+template <typename T, int KP, int CPL>
+cudaError_t launch_uvu_edge(const UvuEdgeParams<T>& p, cudaStream_t s);
+
+template <typename T, int KP, int CPL>
+cudaError_t launch_uvu_src(const UvuSrcParams<T>& p, cudaStream_t s);
+
+template <typename T>
+cudaError_t launch_reduce_slots(const T* part, T* out, int n_slots, long long n, cudaStream_t s);
+
+size_t csr_workspace_bytes(long long n_nodes);
+cudaError_t csr_build(int N, int E, const int* src, const int* dst, int* rowptr, int* senders, int* perm,
+                      void* ws, int* err, cudaStream_t s);
+cudaError_t csr_transpose(int N, int E, const int* rowptr, const int* senders, int* colptr, int* srcedge,
+                          int* srcrecv, void* ws, int* err, cudaStream_t s);
+
+}  // namespace tpc
+
+// Explicit instantiations are split over several compilations of the same file
+// (-DTPC_SET=k builds only set k) so that the build runs in parallel.
+#ifndef TPC_SET
+#define TPC_SET -1
+#endif
+#define TPC_WANT(k) (TPC_SET < 0 || TPC_SET == (k))

@@ -1,0 +1,246 @@
+// Host planner of the tensor-product convolution (Sobek §4.5: the wrapper
+// validates the contract and enumerates valid paths and sparse CG terms; LunaTP
+// §4.2: work is partitioned into tasks over receivers, path groups and channel
+// blocks).
+//
+// Path enumeration (the pages fix no order; this order defines the layout of A):
+// for each input block in the order written, for l2 = 0..L_sh (parity (-1)^l2),
+// for l3 = |l1-l2|..l1+l2, one path to every output block of degree l3 and
+// parity p1 p2 (Sobek §2.2 selection rule), in output order. Output blocks
+// receive the sum over their paths.
+#include "plan.h"
+
+#include <algorithm>
+#include <cctype>
+#include <cmath>
+#include <cstdlib>
+
+#include "cg_host.h"
+#include "tpconv.h"
+
+namespace tpc {
+namespace {
+
+bool parse_irreps(const char* s, std::vector<Block>& out, std::string& msg) {
+  out.clear();
+  if (!s) {
+    msg = "irreps string is NULL";
+    return false;
+  }
+  std::string str(s);
+  size_t pos = 0;
+  int off = 0;
+  while (pos <= str.size()) {
+    size_t end = str.find('+', pos);
+    if (end == std::string::npos) end = str.size();
+    std::string t;
+    for (size_t k = pos; k < end; ++k)
+      if (!std::isspace((unsigned char)str[k])) t.push_back(str[k]);
+    if (t.empty()) {
+      msg = "empty irreps term in '" + str + "'";
+      return false;
+    }
+    int mul = 1;
+    size_t x = t.find('x');
+    std::string ir = t;
+    if (x != std::string::npos) {
+      mul = std::atoi(t.substr(0, x).c_str());
+      ir = t.substr(x + 1);
+      for (size_t k = 0; k < x; ++k)
+        if (!std::isdigit((unsigned char)t[k])) mul = -1;
+    }
+    if (ir.size() < 2 || (ir.back() != 'e' && ir.back() != 'o') || mul <= 0) {
+      msg = "bad irreps term '" + t + "'";
+      return false;
+    }
+    for (size_t k = 0; k + 1 < ir.size(); ++k)
+      if (!std::isdigit((unsigned char)ir[k])) {
+        msg = "bad irreps term '" + t + "'";
+        return false;
+      }
+    const int l = std::atoi(ir.substr(0, ir.size() - 1).c_str());
+    const int p = ir.back() == 'e' ? 1 : -1;
+    out.push_back({mul, l, p, off});
+    off += mul * (2 * l + 1);
+    pos = end + 1;
+  }
+  return !out.empty();
+}
+
+void add_tiles(const std::vector<Block>& blocks, const std::vector<std::vector<int>>& members,
+               const std::vector<HostPath>& paths, int tile_w, bool by_out, std::vector<TileD>& tiles,
+               std::vector<PathD>& plist) {
+  for (size_t b = 0; b < blocks.size(); ++b) {
+    const int pbeg = (int)plist.size();
+    for (int pi : members[b]) {
+      const HostPath& h = paths[pi];
+      PathD d{};
+      d.l1 = (int8_t)h.l1;
+      d.l2 = (int8_t)h.l2;
+      d.l3 = (int8_t)h.l3;
+      d.x_off = h.x_off;
+      d.out_off = h.out_off;
+      d.w_off = (int)h.w_off;
+      d.mul_in = h.mul_in;
+      d.mul_out = h.mul_out;
+      plist.push_back(d);
+    }
+    const int pend = (int)plist.size();
+    const Block& bl = blocks[b];
+    for (int ch0 = 0; ch0 < bl.mul; ch0 += tile_w)
+      tiles.push_back({bl.l, bl.offset, bl.mul, ch0, std::min(tile_w, bl.mul - ch0), pbeg, pend});
+    (void)by_out;
+  }
+}
+
+}  // namespace
+
+int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_radial, int mode,
+              int dtype, Plan& P, std::string& msg) {
+  P = Plan{};
+  if (mode != TP_UVU && mode != TP_UVW) {
+    msg = "mode must be TP_UVU or TP_UVW";
+    return TP_EINVAL;
+  }
+  if (dtype != TP_F32 && dtype != TP_F64) {
+    msg = "dtype must be TP_F32 or TP_F64";
+    return TP_EINVAL;
+  }
+  if (sh_lmax < 0 || n_radial <= 0) {
+    msg = "sh_lmax must be >= 0 and n_radial > 0";
+    return TP_EINVAL;
+  }
+  if (!parse_irreps(irreps_in, P.bin, msg) || !parse_irreps(irreps_out, P.bout, msg)) return TP_EINVAL;
+  P.mode = mode;
+  P.dtype = dtype;
+  P.K = n_radial;
+  P.sh_lmax = sh_lmax;
+  P.dim_y = (sh_lmax + 1) * (sh_lmax + 1);
+  for (auto& b : P.bin) P.c_in += b.mul * (2 * b.l + 1);
+  for (auto& b : P.bout) P.c_out += b.mul * (2 * b.l + 1);
+  long long w = 0;
+  for (size_t i1 = 0; i1 < P.bin.size(); ++i1) {
+    const Block& b1 = P.bin[i1];
+    for (int l2 = 0; l2 <= sh_lmax; ++l2) {
+      const int p2 = (l2 & 1) ? -1 : 1;
+      for (int l3 = std::abs(b1.l - l2); l3 <= b1.l + l2; ++l3) {
+        const int p3 = b1.p * p2;
+        for (size_t io = 0; io < P.bout.size(); ++io) {
+          const Block& bo = P.bout[io];
+          if (bo.l != l3 || bo.p != p3) continue;
+          HostPath h{};
+          h.l1 = b1.l; h.p1 = b1.p; h.l2 = l2; h.p2 = p2; h.l3 = l3; h.p3 = p3;
+          h.i_in = (int)i1; h.i_out = (int)io;
+          h.mul_in = b1.mul; h.mul_out = bo.mul;
+          h.x_off = b1.offset; h.out_off = bo.offset;
+          if (mode == TP_UVU) {
+            if (bo.mul != b1.mul) {
+              msg = "uvu needs equal input and output multiplicity on every path";
+              return TP_EUNSUPPORTED;
+            }
+            h.n_w = b1.mul;
+          } else {
+            h.n_w = (long long)b1.mul * bo.mul;
+          }
+          h.w_off = w;
+          h.nnz = (int)real_cg_sparse(h.l1, h.l2, h.l3).size();
+          w += h.n_w;
+          P.paths.push_back(h);
+          P.lmax = std::max(P.lmax, std::max(h.l1, std::max(h.l2, h.l3)));
+        }
+      }
+    }
+  }
+  P.n_w = w;
+  for (auto& b : P.bin) P.lmax = std::max(P.lmax, b.l);
+  for (auto& b : P.bout) P.lmax = std::max(P.lmax, b.l);
+  P.lmax = std::max(P.lmax, sh_lmax);
+  // limits of the compiled kernels
+  if (P.lmax > kLmax) {
+    msg = "degree " + std::to_string(P.lmax) + " above the kernels' limit " + std::to_string(kLmax);
+    return TP_EUNSUPPORTED;
+  }
+  if (P.K > 16) {
+    msg = "n_radial above 16 is not compiled";
+    return TP_EUNSUPPORTED;
+  }
+  P.KP = P.K <= 8 ? 8 : 16;
+  if ((int)P.paths.size() > kMaxPaths) {
+    msg = "more than " + std::to_string(kMaxPaths) + " paths";
+    return TP_EUNSUPPORTED;
+  }
+  if (P.n_w * (long long)P.K >= (1LL << 31) || P.c_in <= 0 || P.c_out <= 0) {
+    msg = "weight tensor too large for 32-bit indexing";
+    return TP_EUNSUPPORTED;
+  }
+  bool all_even = true;
+  for (auto& b : P.bin) all_even &= (b.mul % 2 == 0);
+  for (auto& b : P.bout) all_even &= (b.mul % 2 == 0);
+  P.CPL = (dtype == TP_F32 && all_even) ? 2 : 1;
+  const int tile_w = 32 * P.CPL;
+  std::vector<std::vector<int>> by_out(P.bout.size()), by_in(P.bin.size());
+  for (size_t k = 0; k < P.paths.size(); ++k) {
+    by_out[P.paths[k].i_out].push_back((int)k);
+    by_in[P.paths[k].i_in].push_back((int)k);
+  }
+  add_tiles(P.bout, by_out, P.paths, tile_w, true, P.out_tiles, P.paths_by_out);
+  add_tiles(P.bin, by_in, P.paths, tile_w, false, P.in_tiles, P.paths_by_in);
+  std::vector<std::vector<int>> all(1);
+  for (size_t k = 0; k < P.paths.size(); ++k) all[0].push_back((int)k);
+  std::vector<TileD> dummy;
+  std::vector<Block> one{{1, 0, 1, 0}};
+  add_tiles(one, all, P.paths, 1, false, dummy, P.paths_canon);
+  if ((int)P.out_tiles.size() > kMaxTiles || (int)P.in_tiles.size() > kMaxTiles) {
+    msg = "more than " + std::to_string(kMaxTiles) + " channel tiles";
+    return TP_EUNSUPPORTED;
+  }
+  return TP_OK;
+}
+
+int uvu_src_slots(const Plan& p, long long n_nodes) {
+  const long long target = 148LL * 24;  // resident warps to aim for on 148 SMs
+  const long long t = std::max<long long>(1, (long long)p.in_tiles.size());
+  long long s = (target + t - 1) / t;
+  s = std::min<long long>(s, std::max<long long>(1, n_nodes));
+  return (int)s;
+}
+
+size_t workspace_bytes(const Plan& p, long long n_nodes, int pass) {
+  const size_t b = p.dtype == TP_F32 ? 4 : 8;
+  size_t bytes = 0;
+  if (p.mode == TP_UVU) {
+    if (pass == 1) bytes = (size_t)uvu_src_slots(p, n_nodes) * p.K * p.n_w * b;
+  }
+  return (bytes + 255) / 256 * 256;
+}
+
+void work_model(const Plan& p, long long N, long long E, int pass, double& flops, double& bytes) {
+  const double b = p.dtype == TP_F32 ? 4.0 : 8.0;
+  double fwd = 0, bwd = 0;
+  for (auto& h : p.paths) {
+    const double d3 = 2 * h.l3 + 1, nnz = h.nnz, K = p.K;
+    if (p.mode == TP_UVU) {
+      const double C = h.mul_in;
+      fwd += 2.0 * E * C * (K + nnz + d3);
+      bwd += 2.0 * E * C * (3 * K + 3 * nnz + 2 * d3);
+    } else {
+      const double ci = h.mul_in, co = h.mul_out;
+      const double e = E * (2 * ci * nnz + 2 * K * ci * d3);
+      const double r = N * 2 * d3 * K * ci * co;
+      fwd += e + r;
+      bwd += r + e + E * (4 * K * ci * d3 + 4 * ci * nnz);
+    }
+  }
+  const double in_b = b * ((double)N * p.c_in + (double)E * p.dim_y + (double)E * p.K + (double)p.K * p.n_w);
+  if (pass == 0) {
+    flops = fwd;
+    bytes = in_b + b * (double)N * p.c_out + 4.0 * E + 4.0 * (N + 1);
+  } else {
+    flops = bwd;
+    bytes = in_b + b * ((double)N * p.c_out + (double)N * p.c_in + (double)E * p.dim_y + (double)E * p.K +
+                        (double)p.K * p.n_w) +
+            12.0 * E + 8.0 * (N + 1);
+  }
+}
+
+}  // namespace tpc

@@ -1,0 +1,53 @@
+// Host-side plan of one tensor-product convolution contract.
+#pragma once
+
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+
+namespace tpc {
+
+struct Block {
+  int mul, l, p, offset;
+};
+
+struct HostPath {
+  int l1, p1, l2, p2, l3, p3;
+  int i_in, i_out, mul_in, mul_out;
+  int x_off, out_off;
+  long long w_off, n_w;
+  int nnz;
+};
+
+struct Plan {
+  int mode = 0;     // 0 uvu, 1 uvw
+  int dtype = 0;    // 0 f32, 1 f64
+  int K = 0, KP = 0, CPL = 1, sh_lmax = 0, lmax = 0;
+  std::vector<Block> bin, bout;
+  std::vector<HostPath> paths;  // canonical enumeration order
+  int c_in = 0, c_out = 0, dim_y = 0;
+  long long n_w = 0;
+  // kernel descriptor tables
+  std::vector<TileD> out_tiles;   // (output block, channel tile), paths_by_out ranges
+  std::vector<PathD> paths_by_out;
+  std::vector<TileD> in_tiles;    // (input block, channel tile), paths_by_in ranges
+  std::vector<PathD> paths_by_in;
+  std::vector<PathD> paths_canon;
+};
+
+// Returns 0 or a negative tp_status; msg receives a human-readable reason.
+int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_radial, int mode,
+              int dtype, Plan& out, std::string& msg);
+
+// Slots of the source pass's A_bar partial buffer (fixed per (plan, N)).
+int uvu_src_slots(const Plan& p, long long n_nodes);
+
+// Bytes of workspace for pass 0 (forward) or 1 (backward) at n_nodes receivers.
+size_t workspace_bytes(const Plan& p, long long n_nodes, int pass);
+
+// Algorithmic flops and compulsory bytes of one pass (0 fwd, 1 bwd).
+void work_model(const Plan& p, long long n_nodes, long long n_edges, int pass, double& flops,
+                double& bytes);
+
+}  // namespace tpc

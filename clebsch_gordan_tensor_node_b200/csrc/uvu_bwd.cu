@@ -1,0 +1,354 @@
+// Channelwise (uvu) first backward of the CG tensor-product convolution.
+//
+// Adjoints (Sobek §3.2; LunaTP Appendix F, Algorithm 2), with m_bar = grad_out:
+//   h_{e,pi,u}      = < m_bar_i[pi], T_{pi,u}(x_j, Y_e) >
+//   A_bar_{q,pi,u}  = sum_e phi_{e,q} h_{e,pi,u}
+//   phi_bar_{e,q}   = sum_{pi,u} A_{q,pi,u} h_{e,pi,u}
+//   x_bar_j         = sum_{e: src=j} sum_{pi,u} w_{e,pi,u} D_x T^* m_bar_i
+//   Y_bar_e         = sum_{pi,u} w_{e,pi,u} D_Y T^* m_bar_i
+// h is consumed where it is formed; no W_bar tensor or edge chunk of it exists
+// (Sobek §3.2, §4.3). Ownership follows Sobek §4.3 and LunaTP §4.4:
+//   * edge pass: one warp per receiver walks its CSR edges; for each edge it
+//     sweeps every path and channel, keeps per-lane partials of phi_bar_e and
+//     Y_bar_e in registers, reduces them across the warp once, and writes them
+//     (each edge has one owner, no cross-edge reduction);
+//   * source pass: one warp per (source j, input block, channel tile) walks the
+//     source-CSR view, accumulates x_bar_j in registers (one fixed order, no
+//     atomics) and, because the same sweep forms h, the A_bar contributions,
+//     which it adds into its own slot of a fixed-size partial buffer
+//     [slots, K, N_w] (independent of E);
+//   * reduce: A_bar = sum over slots in slot order.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace tpc {
+namespace {
+
+constexpr int kDY = (kLmax + 1) * (kLmax + 1);
+
+// ---------------------------------------------------------------- edge pass
+
+template <typename T, int KP, int CPL, int L1, int L2, int L3>
+__device__ __forceinline__ void edge_path(const UvuEdgeParams<T>& p, const PathD& pd, int lane,
+                                          const T* xrow, const T* grow, const T (&ph)[KP],
+                                          const T (&yall)[kDY], T (&gphi)[KP], T (&gY)[kDY]) {
+  using CGp = cgt::CG<L1, L2, L3>;
+  constexpr int D1 = 2 * L1 + 1, D3 = 2 * L3 + 1, Y0 = L2 * L2;
+  const int mul = pd.mul_in;
+  for (int ch0 = 0; ch0 < mul; ch0 += 32 * CPL) {
+    const bool active = ch0 + lane * CPL < mul;
+    const int chl = ch0 + (active ? lane * CPL : 0);
+    T a[KP][CPL], xv[D1][CPL], gv[D3][CPL];
+#pragma unroll
+    for (int q = 0; q < KP; ++q) {
+      if (q < p.K) {
+        load_ch<CPL>(a[q], p.A + (size_t)q * p.n_w + pd.w_off + chl);
+      } else {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) a[q][c] = T(0);
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < D1; ++m) load_ch<CPL>(xv[m], xrow + pd.x_off + m * mul + chl);
+#pragma unroll
+    for (int m = 0; m < D3; ++m) load_ch<CPL>(gv[m], grow + pd.out_off + m * pd.mul_out + chl);
+    if (!active) {
+#pragma unroll
+      for (int m = 0; m < D1; ++m)
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) xv[m][c] = T(0);
+    }
+    T w[CPL], h[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      w[c] = ph[0] * a[0][c];
+#pragma unroll
+      for (int q = 1; q < KP; ++q) w[c] = fma(ph[q], a[q][c], w[c]);
+      h[c] = T(0);
+    }
+    static_for<CGp::npair>([&](auto P) {
+      constexpr int Pi = decltype(P)::value;
+      constexpr Pair pr = CGp::pair[Pi];
+      const T cy = pair_coef<T, CGp, Pi>(yall + Y0);
+      T z = T(0);
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        const T xg = xv[pr.m1][c] * gv[pr.m3][c];
+        h[c] = fma(cy, xg, h[c]);
+        z = fma(w[c], xg, z);
+      }
+      // Y_bar[m2] += c * sum_u w x[m1] m_bar[m3]
+      static_for<pr.n>([&](auto t) {
+        constexpr Term tm = CGp::term[pr.start + decltype(t)::value];
+        gY[Y0 + tm.m2] = fma(T(tm.c), z, gY[Y0 + tm.m2]);
+      });
+    });
+#pragma unroll
+    for (int q = 0; q < KP; ++q)
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) gphi[q] = fma(a[q][c], h[c], gphi[q]);
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <typename T, int KP, int CPL>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+uvu_edge_kernel(const __grid_constant__ UvuEdgeParams<T> p) {
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  if (i >= p.N) return;
+  int e0 = ldg(p.rowptr + i), e1 = ldg(p.rowptr + i + 1);
+  if (e0 < 0 || e1 < e0 || e1 > p.E) {
+    raise_error(p.err, kErrCsr);
+    return;
+  }
+  const T* grow = p.gout + (size_t)i * p.c_out;
+  for (int e = e0; e < e1; ++e) {
+    const int j = ldg(p.senders + e);
+    T gphi[KP], gY[kDY];
+#pragma unroll
+    for (int q = 0; q < KP; ++q) gphi[q] = T(0);
+#pragma unroll
+    for (int m = 0; m < kDY; ++m) gY[m] = T(0);
+    if ((unsigned)j < (unsigned)p.N) {
+      T ph[KP], yall[kDY];
+      load_phi<KP>(ph, p.phi + (size_t)e * p.K, p.K);
+#pragma unroll
+      for (int m = 0; m < kDY; ++m) yall[m] = m < p.dim_y ? ldg(p.Y + (size_t)e * p.dim_y + m) : T(0);
+      const T* xrow = p.x + (size_t)j * p.c_in;
+      for (int pi = 0; pi < p.n_paths; ++pi) {
+        const PathD& pd = p.paths[pi];
+        dispatch_l(pd.l1, [&](auto A1) {
+          constexpr int L1 = decltype(A1)::value;
+          dispatch_l2l3<L1>(pd.l2, pd.l3, [&](auto A2, auto A3) {
+            edge_path<T, KP, CPL, L1, decltype(A2)::value, decltype(A3)::value>(
+                p, pd, lane, xrow, grow, ph, yall, gphi, gY);
+          });
+        });
+      }
+    } else {
+      raise_error(p.err, kErrIndex);
+    }
+    // one reduction per edge; lane 0 writes
+#pragma unroll
+    for (int q = 0; q < KP; ++q) {
+      if (q < p.K) {
+        const T v = warp_sum(gphi[q]);
+        if (lane == 0) p.gphi[(size_t)e * p.K + q] = v;
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < kDY; ++m) {
+      if (m < p.dim_y) {
+        const T v = warp_sum(gY[m]);
+        if (lane == 0) p.gY[(size_t)e * p.dim_y + m] = v;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- source pass
+
+template <typename T, int KP, int CPL, int L1, int L2, int L3>
+__device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& pd, int slot,
+                                         int chl, bool active, int k0, int k1,
+                                         const T (&xs)[2 * L1 + 1][CPL], T (&gx)[2 * L1 + 1][CPL]) {
+  using CGp = cgt::CG<L1, L2, L3>;
+  constexpr int D1 = 2 * L1 + 1, D2 = 2 * L2 + 1, D3 = 2 * L3 + 1;
+  T a[KP][CPL], ab[KP][CPL];
+#pragma unroll
+  for (int q = 0; q < KP; ++q) {
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) ab[q][c] = T(0);
+    if (q < p.K) {
+      load_ch<CPL>(a[q], p.A + (size_t)q * p.n_w + pd.w_off + chl);
+    } else {
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) a[q][c] = T(0);
+    }
+  }
+  const int mo = pd.mul_out;
+  for (int k = k0; k < k1; ++k) {
+    const int e = ldg(p.srcedge + k);
+    const int i = ldg(p.srcrecv + k);
+    if ((unsigned)e >= (unsigned)p.E || (unsigned)i >= (unsigned)p.N) {
+      raise_error(p.err, kErrIndex);
+      continue;
+    }
+    T ph[KP], y[D2], gv[D3][CPL];
+    load_phi<KP>(ph, p.phi + (size_t)e * p.K, p.K);
+#pragma unroll
+    for (int m = 0; m < D2; ++m) y[m] = ldg(p.Y + (size_t)e * p.dim_y + L2 * L2 + m);
+    const T* gr = p.gout + (size_t)i * p.c_out + pd.out_off + chl;
+#pragma unroll
+    for (int m = 0; m < D3; ++m) load_ch<CPL>(gv[m], gr + m * mo);
+    T w[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      w[c] = ph[0] * a[0][c];
+#pragma unroll
+      for (int q = 1; q < KP; ++q) w[c] = fma(ph[q], a[q][c], w[c]);
+    }
+    // t'[m1] = sum_{m3} cY[m1][m3] m_bar[m3]   (D_x T^* applied to m_bar)
+    T tp[D1][CPL];
+    static_for<CGp::npair>([&](auto P) {
+      constexpr int Pi = decltype(P)::value;
+      constexpr Pair pr = CGp::pair[Pi];
+      const T cy = pair_coef<T, CGp, Pi>(y);
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        if constexpr (first_m1<CGp>(Pi))
+          tp[pr.m1][c] = cy * gv[pr.m3][c];
+        else
+          tp[pr.m1][c] = fma(cy, gv[pr.m3][c], tp[pr.m1][c]);
+      }
+    });
+    T h[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) h[c] = T(0);
+    static_for<D1>([&](auto M) {
+      constexpr int m1 = decltype(M)::value;
+      if constexpr (has_m1<CGp>(m1)) {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          gx[m1][c] = fma(w[c], tp[m1][c], gx[m1][c]);
+          h[c] = fma(xs[m1][c], tp[m1][c], h[c]);
+        }
+      }
+    });
+#pragma unroll
+    for (int q = 0; q < KP; ++q)
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) ab[q][c] = fma(ph[q], h[c], ab[q][c]);
+  }
+  if (active && k1 > k0) {
+#pragma unroll
+    for (int q = 0; q < KP; ++q) {
+      if (q < p.K) {
+        T* dst = p.apart + ((size_t)slot * p.K + q) * p.n_w + pd.w_off + chl;
+        T v[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) v[c] = dst[c] + ab[q][c];
+        store_ch<CPL>(dst, v);
+      }
+    }
+  }
+}
+
+template <typename T, int KP, int CPL, int L1>
+__device__ __forceinline__ void src_tile(const UvuSrcParams<T>& p, const TileD& tl, int slot, int lane) {
+  constexpr int D1 = 2 * L1 + 1;
+  const bool active = lane * CPL < tl.nch;
+  const int chl = tl.ch0 + (active ? lane * CPL : 0);
+  for (int j = slot; j < p.N; j += p.n_slots) {
+    int k0 = ldg(p.colptr + j), k1 = ldg(p.colptr + j + 1);
+    if (k0 < 0 || k1 < k0 || k1 > p.E) {
+      raise_error(p.err, kErrCsr);
+      k1 = k0;
+    }
+    T xs[D1][CPL], gx[D1][CPL];
+    const T* xr = p.x + (size_t)j * p.c_in + tl.off + chl;
+#pragma unroll
+    for (int m = 0; m < D1; ++m) {
+      load_ch<CPL>(xs[m], xr + m * tl.mul);
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) gx[m][c] = T(0);
+    }
+    for (int pi = tl.pbeg; pi < tl.pend; ++pi) {
+      const PathD& pd = p.paths[pi];
+      dispatch_l2l3<L1>(pd.l2, pd.l3, [&](auto A2, auto A3) {
+        src_path<T, KP, CPL, L1, decltype(A2)::value, decltype(A3)::value>(p, pd, slot, chl, active,
+                                                                           k0, k1, xs, gx);
+      });
+    }
+    if (active) {
+      T* o = p.gx + (size_t)j * p.c_in + tl.off + chl;
+#pragma unroll
+      for (int m = 0; m < D1; ++m) store_ch<CPL>(o + m * tl.mul, gx[m]);
+    }
+  }
+}
+
+template <typename T, int KP, int CPL>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+uvu_src_kernel(const __grid_constant__ UvuSrcParams<T> p) {
+  const int lane = threadIdx.x & 31;
+  const int wid = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  if (wid >= p.n_slots * p.n_tiles) return;
+  const int slot = wid / p.n_tiles;
+  const TileD& tl = p.tiles[wid % p.n_tiles];
+  dispatch_l(tl.l, [&](auto L) { src_tile<T, KP, CPL, decltype(L)::value>(p, tl, slot, lane); });
+}
+
+template <typename T>
+__global__ void reduce_slots_kernel(const T* __restrict__ part, T* __restrict__ out, int n_slots,
+                                    long long n) {
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= n) return;
+  T s = T(0);
+  for (int k = 0; k < n_slots; ++k) s += part[(size_t)k * n + t];
+  out[t] = s;
+}
+
+}  // namespace
+
+template <typename T, int KP, int CPL>
+cudaError_t launch_uvu_edge(const UvuEdgeParams<T>& p, cudaStream_t s) {
+  if (p.N == 0) return cudaSuccess;
+  const int blocks = (p.N + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  uvu_edge_kernel<T, KP, CPL><<<blocks, kWarpsPerBlock * 32, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T, int KP, int CPL>
+cudaError_t launch_uvu_src(const UvuSrcParams<T>& p, cudaStream_t s) {
+  cudaError_t err = cudaMemsetAsync(p.apart, 0, sizeof(T) * (size_t)p.n_slots * p.K * p.n_w, s);
+  if (err != cudaSuccess) return err;
+  const long long warps = (long long)p.n_slots * p.n_tiles;
+  if (warps == 0 || p.N == 0) return cudaSuccess;
+  const long long blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  uvu_src_kernel<T, KP, CPL><<<(unsigned)blocks, kWarpsPerBlock * 32, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_reduce_slots(const T* part, T* out, int n_slots, long long n, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  reduce_slots_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(part, out, n_slots, n);
+  return cudaGetLastError();
+}
+
+#define TPC_INST(T, KP, CPL)                                                                   \
+  template cudaError_t launch_uvu_edge<T, KP, CPL>(const UvuEdgeParams<T>&, cudaStream_t);     \
+  template cudaError_t launch_uvu_src<T, KP, CPL>(const UvuSrcParams<T>&, cudaStream_t);
+#if TPC_WANT(0)
+TPC_INST(float, 8, 1)
+#endif
+#if TPC_WANT(1)
+TPC_INST(float, 8, 2)
+#endif
+#if TPC_WANT(2)
+TPC_INST(float, 16, 1)
+#endif
+#if TPC_WANT(3)
+TPC_INST(float, 16, 2)
+#endif
+#if TPC_WANT(4)
+TPC_INST(double, 8, 1)
+#endif
+#if TPC_WANT(5)
+TPC_INST(double, 16, 1)
+#endif
+#undef TPC_INST
+#if TPC_WANT(0)
+template cudaError_t launch_reduce_slots<float>(const float*, float*, int, long long, cudaStream_t);
+template cudaError_t launch_reduce_slots<double>(const double*, double*, int, long long, cudaStream_t);
+#endif
+
+}  // namespace tpc

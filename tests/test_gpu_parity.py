@@ -1,0 +1,105 @@
+"""GPU parity of the library against the oracle, through the C ABI.
+
+Bar (from the operator's numerics): per output tensor
+max_k |gpu_k - oracle_k| / max_k |oracle_k| <= 1e-4 (fp32) and <= 1e-10 (fp64);
+CSR, permutation and source views bit-exact; two runs bitwise identical
+(Sobek §5.1 double-peer determinism).
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import TOL, GpuRun, plan_for, problem, rel_err, workload
+from inputs import CONFIGS
+from oracle import conv as oconv
+from oracle import csr as ocsr
+
+pytestmark = pytest.mark.gpu
+
+# (config, nodes or None for the full workload): small enough for the oracle
+CASES = [(1, None), (3, None), (2, 384), (4, 1500)]
+
+
+def _check_csr(run):
+    wl = run.wl
+    rp, snd, perm = ocsr.build(wl.n_nodes, wl.src, wl.dst)
+    assert np.array_equal(run.rowptr.cpu().numpy(), rp)
+    assert np.array_equal(run.senders.cpu().numpy(), snd)
+    assert np.array_equal(run.perm.cpu().numpy(), perm)
+    cp, se, sr = ocsr.transpose(wl.n_nodes, rp, snd)
+    assert np.array_equal(run.colptr.cpu().numpy(), cp)
+    assert np.array_equal(run.srcedge.cpu().numpy(), se)
+    assert np.array_equal(run.srcrecv.cpu().numpy(), sr)
+
+
+@pytest.mark.parametrize("cid,n", CASES)
+def test_forward_backward_parity(cid, n):
+    c = CONFIGS[cid]
+    wl = workload(cid, n_nodes=n)
+    run = GpuRun(plan_for(cid), wl)
+    _check_csr(run)
+    pr = problem(cid)
+    out = run.forward()
+    want = oconv.forward(pr, wl.x, wl.Y, wl.phi, wl.A, wl.src, wl.dst, wl.n_nodes)
+    assert rel_err(out.cpu().numpy(), want) <= TOL[c.dtype]
+    gx, gY, gphi, gA = run.backward()
+    ox, oY, ophi, oA = oconv.backward(pr, wl.x, wl.Y, wl.phi, wl.A, wl.src, wl.dst, wl.grad_out,
+                                      wl.n_nodes)
+    assert rel_err(gx.cpu().numpy(), ox) <= TOL[c.dtype]
+    assert rel_err(run.to_coo(gY), oY) <= TOL[c.dtype]
+    assert rel_err(run.to_coo(gphi), ophi) <= TOL[c.dtype]
+    assert rel_err(gA.cpu().numpy(), oA) <= TOL[c.dtype]
+    assert tpc_error() == 0
+
+
+def tpc_error():
+    import clebsch_gordan_tensor_node_b200 as tpc
+    return tpc.tp_get_device_error()
+
+
+@pytest.mark.parametrize("cid", [1, 4])
+def test_bitwise_reproducible(cid):
+    wl = workload(cid, n_nodes=None if cid == 1 else 1200)
+    run = GpuRun(plan_for(cid), wl)
+    a = run.forward().clone()
+    ga = [t.clone() for t in run.backward()]
+    b = run.forward()
+    gb = run.backward()
+    assert torch.equal(a, b)
+    for u, v in zip(ga, gb):
+        assert torch.equal(u, v)
+
+
+@pytest.mark.parametrize("cid", [2, 4])
+def test_full_size_sampled(cid):
+    """Full-size workload in the benchmark's launch configuration: forward rows of
+    sampled receivers, grad_phi/grad_Y of their edges and grad_x of sampled
+    sources against the oracle restricted to those edges; grad_A through the
+    adjoint identity <grad_A, V> = <grad_out, forward(A = V)>, which holds at any
+    size because the operator is linear in A."""
+    c = CONFIGS[cid]
+    wl = workload(cid)
+    run = GpuRun(plan_for(cid), wl)
+    pr = problem(cid)
+    rng = np.random.default_rng(100 + cid)
+    recv = rng.choice(wl.n_nodes, 48, replace=False)
+    sel = np.isin(wl.dst, recv)
+    out = run.forward().cpu().numpy()
+    want = oconv.forward(pr, wl.x, wl.Y[sel], wl.phi[sel], wl.A, wl.src[sel], wl.dst[sel], wl.n_nodes)
+    assert rel_err(out[recv], want[recv]) <= TOL[c.dtype]
+    if not c.backward:
+        return
+    gx, gY, gphi, gA = run.backward()
+    ox, oY, ophi, _ = oconv.backward(pr, wl.x, wl.Y[sel], wl.phi[sel], wl.A, wl.src[sel], wl.dst[sel],
+                                     wl.grad_out, wl.n_nodes)
+    assert rel_err(run.to_coo(gY)[sel], oY) <= TOL[c.dtype]
+    assert rel_err(run.to_coo(gphi)[sel], ophi) <= TOL[c.dtype]
+    srcs = rng.choice(wl.n_nodes, 32, replace=False)
+    ssel = np.isin(wl.src, srcs)
+    ox, *_ = oconv.backward(pr, wl.x, wl.Y[ssel], wl.phi[ssel], wl.A, wl.src[ssel], wl.dst[ssel],
+                            wl.grad_out, wl.n_nodes)
+    assert rel_err(gx.cpu().numpy()[srcs], ox[srcs]) <= TOL[c.dtype]
+    V = torch.randn_like(run.A)
+    lhs = float((gA.double() * V.double()).sum())
+    rhs = float((run.gout.double() * run.forward(A=V).double()).sum())
+    assert abs(lhs - rhs) <= 1e-4 * (abs(gA.double()).sum().item() * V.abs().max().item())
