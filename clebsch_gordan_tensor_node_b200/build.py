@@ -25,7 +25,7 @@ CG_LMAX = 6
 
 # translation units and how many instantiation sets each one is split into
 UNITS = {
-    "uvu_fwd.cu": 6,
+    "uvu_fwd.cu": 9,
     "uvu_bwd.cu": 6,
     "csr.cu": 1,
     "api.cu": 1,

@@ -78,10 +78,32 @@ cudaError_t dispatch_kc(const Plan& P, const Prm& prm, cudaStream_t s) {
   return cudaErrorInvalidValue;
 }
 
-template <typename T, int KP, int CPL>
-struct FwdL {
-  static cudaError_t run(const UvuFwdParams<T>& p, cudaStream_t s) { return launch_uvu_fwd<T, KP, CPL>(p, s); }
-};
+template <typename T, int KP, int CPL, bool Full>
+cudaError_t fwd_prof(const Plan& P, const UvuFwdParams<T>& p, cudaStream_t s) {
+  switch (P.prof) {
+    case 0: return launch_uvu_fwd<T, KP, CPL, 2, 2, 2>(p, s);
+    case 1: return launch_uvu_fwd<T, KP, CPL, 1, 3, 3>(p, s);
+    case 2: return launch_uvu_fwd<T, KP, CPL, 3, 3, 3>(p, s);
+    default:
+      if constexpr (Full) return launch_uvu_fwd<T, KP, CPL, 4, 4, 4>(p, s);
+      return cudaErrorInvalidValue;
+  }
+}
+
+// Mirrors the instantiation list of uvu_fwd.cu.
+template <typename T>
+cudaError_t fwd_dispatch(const Plan& P, const UvuFwdParams<T>& p, cudaStream_t s) {
+  constexpr bool f32 = std::is_same<T, float>::value;
+  if (P.KP == 8) {
+    if (P.fwd_CPL == 1) return fwd_prof<T, 8, 1, true>(P, p, s);
+    if (P.fwd_CPL == 2) return fwd_prof<T, 8, 2, f32>(P, p, s);
+  } else {
+    if (P.fwd_CPL == 1) return fwd_prof<T, 16, 1, true>(P, p, s);
+    if (P.fwd_CPL == 2) return fwd_prof<T, 16, 2, f32>(P, p, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
 template <typename T, int KP, int CPL>
 struct EdgeL {
   static cudaError_t run(const UvuEdgeParams<T>& p, cudaStream_t s) { return launch_uvu_edge<T, KP, CPL>(p, s); }
@@ -99,8 +121,11 @@ int forward_uvu(const Plan& P, const void* x, const void* Y, const void* phi, co
   prm.rowptr = rowptr; prm.senders = senders; prm.out = (T*)out; prm.err = err;
   prm.N = N; prm.E = E; prm.K = P.K; prm.c_in = P.c_in; prm.c_out = P.c_out; prm.dim_y = P.dim_y;
   prm.n_w = (int)P.n_w;
+  prm.cy_stride = P.cy_stride;
+  prm.chunk = P.fwd_chunk;
+  prm.warp_smem = P.fwd_warp_smem;
   copy_tables(prm, P.out_tiles, P.paths_by_out);
-  cudaError_t e = dispatch_kc<T, FwdL>(P, prm, s);
+  cudaError_t e = fwd_dispatch<T>(P, prm, s);
   return e == cudaSuccess ? TP_OK : cuda_fail(e, "uvu forward launch");
 }
 

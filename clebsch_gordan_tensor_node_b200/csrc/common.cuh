@@ -31,6 +31,7 @@ struct PathD {          // one coupling path (l1, l2) -> l3
   int w_off;            // first column of the path in A
   int mul_in;
   int mul_out;
+  int cy_off;           // forward: first cY slot of the path in a staged edge row
 };
 
 struct TileD {          // one channel tile of one irrep block
@@ -52,6 +53,9 @@ struct UvuFwdParams {
   T* out; int* err;
   int N, E, K, c_in, c_out, dim_y, n_w;
   int n_tiles;
+  int cy_stride;              // cY slots per staged edge (max over tiles, padded)
+  int chunk;                  // edges staged per warp at a time (<= 32)
+  int warp_smem;              // bytes of shared memory per warp
   TileD tiles[kMaxTiles];     // one per (output block, channel tile)
   PathD paths[kMaxPaths];     // grouped by output block
 };
@@ -134,11 +138,11 @@ __device__ __forceinline__ T pair_coef(const T* y) {
 }
 
 // Call f(integral_constant<L1>, integral_constant<L2>) for the runtime (l1, l2)
-// among the pairs that can couple into L3.
-template <int L3, typename F>
+// among the pairs that can couple into L3 (degrees up to LM).
+template <int L3, int L1M = kLmax, int L2M = kLmax, typename F>
 __device__ __forceinline__ void dispatch_l1l2(int l1, int l2, F&& f) {
-  static_for<kLmax + 1>([&](auto A1) {
-    static_for<kLmax + 1>([&](auto A2) {
+  static_for<L1M + 1>([&](auto A1) {
+    static_for<L2M + 1>([&](auto A2) {
       constexpr int a = decltype(A1)::value, b = decltype(A2)::value;
       if constexpr (triangle(a, b, L3)) {
         if (l1 == a && l2 == b) f(A1, A2);
@@ -148,10 +152,10 @@ __device__ __forceinline__ void dispatch_l1l2(int l1, int l2, F&& f) {
 }
 
 // Same for (l2, l3) at fixed L1.
-template <int L1, typename F>
+template <int L1, int LM = kLmax, typename F>
 __device__ __forceinline__ void dispatch_l2l3(int l2, int l3, F&& f) {
-  static_for<kLmax + 1>([&](auto A2) {
-    static_for<kLmax + 1>([&](auto A3) {
+  static_for<LM + 1>([&](auto A2) {
+    static_for<LM + 1>([&](auto A3) {
       constexpr int b = decltype(A2)::value, c = decltype(A3)::value;
       if constexpr (triangle(L1, b, c)) {
         if (l2 == b && l3 == c) f(A2, A3);
@@ -161,9 +165,9 @@ __device__ __forceinline__ void dispatch_l2l3(int l2, int l3, F&& f) {
 }
 
 // Same for one degree.
-template <typename F>
+template <int LM = kLmax, typename F>
 __device__ __forceinline__ void dispatch_l(int l, F&& f) {
-  static_for<kLmax + 1>([&](auto A) {
+  static_for<LM + 1>([&](auto A) {
     if (l == decltype(A)::value) f(A);
   });
 }

@@ -7,7 +7,7 @@
 
 namespace tpc {
 
-template <typename T, int KP, int CPL>
+template <typename T, int KP, int CPL, int L1M, int L2M, int L3M>
 cudaError_t launch_uvu_fwd(const UvuFwdParams<T>& p, cudaStream_t s);
 
 template <typename T, int KP, int CPL>

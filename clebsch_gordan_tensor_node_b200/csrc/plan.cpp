@@ -67,8 +67,10 @@ bool parse_irreps(const char* s, std::vector<Block>& out, std::string& msg) {
   return !out.empty();
 }
 
+// Appends, for every block, its member paths to plist and one tile per run of
+// tile_w channels to tiles (each tile refers to the block's path range).
 void add_tiles(const std::vector<Block>& blocks, const std::vector<std::vector<int>>& members,
-               const std::vector<HostPath>& paths, int tile_w, bool by_out, std::vector<TileD>& tiles,
+               const std::vector<HostPath>& paths, int tile_w, std::vector<TileD>& tiles,
                std::vector<PathD>& plist) {
   for (size_t b = 0; b < blocks.size(); ++b) {
     const int pbeg = (int)plist.size();
@@ -89,7 +91,6 @@ void add_tiles(const std::vector<Block>& blocks, const std::vector<std::vector<i
     const Block& bl = blocks[b];
     for (int ch0 = 0; ch0 < bl.mul; ch0 += tile_w)
       tiles.push_back({bl.l, bl.offset, bl.mul, ch0, std::min(tile_w, bl.mul - ch0), pbeg, pend});
-    (void)by_out;
   }
 }
 
@@ -174,26 +175,71 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
     return TP_EUNSUPPORTED;
   }
   bool all_even = true;
-  for (auto& b : P.bin) all_even &= (b.mul % 2 == 0);
-  for (auto& b : P.bout) all_even &= (b.mul % 2 == 0);
+  int min_mul = 1 << 30;
+  for (const auto* v : {&P.bin, &P.bout})
+    for (auto& b : *v) {
+      all_even &= (b.mul % 2 == 0);
+      min_mul = std::min(min_mul, b.mul);
+    }
+  // backward kernels: 1 or 2 channels per lane (fp32), 1 (fp64)
   P.CPL = (dtype == TP_F32 && all_even) ? 2 : 1;
-  const int tile_w = 32 * P.CPL;
+  // forward: vector width by dtype and block width (every access CPL-aligned);
+  // 4 channels per lane measured slower than 2 on the 128-channel workload
+  if (dtype == TP_F32)
+    P.fwd_CPL = all_even ? 2 : 1;
+  else
+    P.fwd_CPL = (all_even && min_mul >= 64) ? 2 : 1;
+  // degree profile of the forward kernel: (max input l, sh_lmax, max output l)
+  // bounded by one of the compiled profiles
+  int lin = 0, lout = 0;
+  for (auto& b : P.bin) lin = std::max(lin, b.l);
+  for (auto& b : P.bout) lout = std::max(lout, b.l);
+  const int profs[4][3] = {{2, 2, 2}, {1, 3, 3}, {3, 3, 3}, {4, 4, 4}};
+  for (int k = 0; k < 4; ++k)
+    if (lin <= profs[k][0] && sh_lmax <= profs[k][1] && lout <= profs[k][2]) {
+      P.prof = k;
+      break;
+    }
+  // instantiated combinations (uvu_fwd.cu): fp64 with 2 channels per lane only
+  // with profiles 0-2
+  if (dtype == TP_F64 && P.fwd_CPL == 2 && P.prof == 3) P.fwd_CPL = 1;
   std::vector<std::vector<int>> by_out(P.bout.size()), by_in(P.bin.size());
   for (size_t k = 0; k < P.paths.size(); ++k) {
     by_out[P.paths[k].i_out].push_back((int)k);
     by_in[P.paths[k].i_in].push_back((int)k);
   }
-  add_tiles(P.bout, by_out, P.paths, tile_w, true, P.out_tiles, P.paths_by_out);
-  add_tiles(P.bin, by_in, P.paths, tile_w, false, P.in_tiles, P.paths_by_in);
+  add_tiles(P.bout, by_out, P.paths, 32 * P.fwd_CPL, P.out_tiles, P.paths_by_out);
+  add_tiles(P.bin, by_in, P.paths, 32 * P.CPL, P.in_tiles, P.paths_by_in);
   std::vector<std::vector<int>> all(1);
   for (size_t k = 0; k < P.paths.size(); ++k) all[0].push_back((int)k);
-  std::vector<TileD> dummy;
+  std::vector<TileD> unused;
   std::vector<Block> one{{1, 0, 1, 0}};
-  add_tiles(one, all, P.paths, 1, false, dummy, P.paths_canon);
+  add_tiles(one, all, P.paths, 1, unused, P.paths_canon);
   if ((int)P.out_tiles.size() > kMaxTiles || (int)P.in_tiles.size() > kMaxTiles) {
     msg = "more than " + std::to_string(kMaxTiles) + " channel tiles";
     return TP_EUNSUPPORTED;
   }
+  // forward staging: per output block, the cY slots of its paths, each padded
+  // to a 16-byte vector so that the kernel reads them with 16-byte loads
+  const int bsz = dtype == TP_F32 ? 4 : 8, vw = 16 / bsz;
+  P.cy_stride = vw;
+  for (const TileD& t : P.out_tiles) {
+    int off = 0;
+    for (int k = t.pbeg; k < t.pend; ++k) {
+      PathD& d = P.paths_by_out[k];
+      auto e = real_cg_sparse(d.l1, d.l2, d.l3);
+      std::vector<std::pair<int, int>> pairs;
+      for (auto& q : e) pairs.emplace_back(q.m1, q.m3);
+      std::sort(pairs.begin(), pairs.end());
+      pairs.erase(std::unique(pairs.begin(), pairs.end()), pairs.end());
+      d.cy_off = off;
+      off += ((int)pairs.size() + vw - 1) / vw * vw;
+    }
+    P.cy_stride = std::max(P.cy_stride, off);
+  }
+  P.fwd_chunk = std::max(1, std::min(32, (20 * 1024) / (P.cy_stride * bsz)));
+  P.fwd_warp_smem = 32 * 4 + 32 * P.KP * bsz + P.fwd_chunk * P.cy_stride * bsz;
+  P.fwd_warp_smem = (P.fwd_warp_smem + 15) / 16 * 16;
   return TP_OK;
 }
 

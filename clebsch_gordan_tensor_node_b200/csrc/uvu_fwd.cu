@@ -9,25 +9,78 @@
 // (receiver i, output block g, tile of 32*CPL channels), lanes own CPL adjacent
 // channels, the receiver's incoming edges (CSR by receiver) form the inner loop,
 // and the output accumulators of block g stay in registers until the single
-// store. Paths into g run one after another (outer loop); their A values live in
-// registers for the whole edge traversal of that path.
+// store. Paths into g run one after another; their A values live in registers
+// for the whole edge traversal of that path.
 //
-// Per edge and path the CG contraction is split into an edge-uniform part and a
-// per-channel part: cY[m1][m3] = sum_{m2} c[m1,m2,m3] Y[m2] (a few FMAs shared by
-// the warp's CPL channels) and acc[m3] += cY[m1][m3] * (w x[m1]) over the
-// non-zero (m1, m3) pairs only; coefficients and indices are compile-time
-// constants (LunaTP §4.3, sparse expansion).
+// The CG contraction is split (Sobek §4.2, Eq. 32) into an edge-uniform part
+// cY[m1][m3] = sum_{m2} c[m1,m2,m3] Y[m2] and a per-channel part
+// acc[m3] += cY[m1][m3] * (w x[m1]) over the non-zero (m1, m3) pairs; the
+// coefficients and pair structure are compile-time constants (LunaTP §4.3).
+// Edges are processed in chunks of up to 32: first each lane takes one edge of
+// the chunk and writes its sender, radial row and the cY values of every path
+// of the tile into the warp's shared-memory slice; then the warp sweeps the
+// chunk once per path, reading those values as broadcasts while the gather of
+// the next sender's x row is already in flight.
+//
+// Task order: windows of kWin receivers; inside a window all receivers of one
+// tile come first, so the warps of a CTA run the same code on neighbouring
+// receivers, and the window's x rows are re-read from L2 by the other tiles.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace tpc {
 namespace {
 
-template <typename T, int KP, int CPL, int L1, int L2, int L3>
-__device__ __forceinline__ void fwd_path(const UvuFwdParams<T>& p, const PathD& pd, int chl,
-                                         int e0, int e1, T (&acc)[2 * L3 + 1][CPL]) {
+constexpr int kWin = 16;
+
+template <typename T>
+struct FwdSmem {
+  int* j;
+  T* phi;
+  T* cy;
+};
+
+template <typename T, int KP>
+__device__ __forceinline__ FwdSmem<T> fwd_smem(const UvuFwdParams<T>& p, int warp) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  unsigned char* base = smem_raw + (size_t)warp * p.warp_smem;
+  FwdSmem<T> s;
+  s.j = reinterpret_cast<int*>(base);
+  s.phi = reinterpret_cast<T*>(base + 32 * sizeof(int));
+  s.cy = s.phi + 32 * KP;
+  return s;
+}
+
+// Stage the cY values of one path for the calling lane's edge.
+template <typename T, int L1, int L2, int L3>
+__device__ __forceinline__ void stage_cy(const T* yrow, T* dst) {
   using CGp = cgt::CG<L1, L2, L3>;
-  constexpr int D1 = 2 * L1 + 1, D2 = 2 * L2 + 1, D3 = 2 * L3 + 1;
+  T y[2 * L2 + 1];
+#pragma unroll
+  for (int m = 0; m < 2 * L2 + 1; ++m) y[m] = ldg(yrow + L2 * L2 + m);
+  static_for<CGp::npair>([&](auto P) { dst[decltype(P)::value] = pair_coef<T, CGp, decltype(P)::value>(y); });
+}
+
+// 16-byte shared-memory load of VW scalars.
+template <typename T>
+__device__ __forceinline__ void lds16(T* v, const T* src) {
+  if constexpr (sizeof(T) == 4) {
+    const float4 t = *reinterpret_cast<const float4*>(src);
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+  } else {
+    const double2 t = *reinterpret_cast<const double2*>(src);
+    v[0] = t.x; v[1] = t.y;
+  }
+}
+
+template <typename T, int KP, int CPL, int L1, int L2, int L3>
+__device__ __forceinline__ void fwd_path(const UvuFwdParams<T>& p, const PathD& pd, const FwdSmem<T>& s,
+                                         int n, int chl, T (&acc)[2 * L3 + 1][CPL]) {
+  using CGp = cgt::CG<L1, L2, L3>;
+  constexpr int D1 = 2 * L1 + 1, D3 = 2 * L3 + 1, NP = CGp::npair;
+  constexpr int VW = sizeof(T) == 4 ? 4 : 2;           // scalars per 16-byte shared load
+  // double-buffer the x gather only while the buffer stays small
+  constexpr bool kPrefetch = D1 * CPL * sizeof(T) <= 48;
   T a[KP][CPL];
 #pragma unroll
   for (int q = 0; q < KP; ++q) {
@@ -39,23 +92,31 @@ __device__ __forceinline__ void fwd_path(const UvuFwdParams<T>& p, const PathD& 
     }
   }
   const T* xb = p.x + pd.x_off + chl;
-  const T* yb = p.Y + L2 * L2;
   const int mul = pd.mul_in;
-  for (int e = e0; e < e1; ++e) {
-    const int j = ldg(p.senders + e);
-    if ((unsigned)j >= (unsigned)p.N) {
-      raise_error(p.err, kErrIndex);
-      continue;
-    }
-    T ph[KP];
-    load_phi<KP>(ph, p.phi + (size_t)e * p.K, p.K);
-    T y[D2];
-#pragma unroll
-    for (int m = 0; m < D2; ++m) y[m] = ldg(yb + (size_t)e * p.dim_y + m);
-    T xv[D1][CPL];
-    const T* xr = xb + (size_t)j * p.c_in;
+  T xv[D1][CPL];
+  if (kPrefetch && n > 0) {
+    const T* xr = xb + (size_t)s.j[0] * p.c_in;
 #pragma unroll
     for (int m = 0; m < D1; ++m) load_ch<CPL>(xv[m], xr + m * mul);
+  }
+  for (int k = 0; k < n; ++k) {
+    T xn[kPrefetch ? D1 : 1][CPL];
+    if constexpr (kPrefetch) {
+      // gather of the next edge's x row, in flight during this edge's arithmetic
+      if (k + 1 < n) {
+        const T* xr = xb + (size_t)s.j[k + 1] * p.c_in;
+#pragma unroll
+        for (int m = 0; m < D1; ++m) load_ch<CPL>(xn[m], xr + m * mul);
+      }
+    } else {
+      const T* xr = xb + (size_t)s.j[k] * p.c_in;
+#pragma unroll
+      for (int m = 0; m < D1; ++m) load_ch<CPL>(xv[m], xr + m * mul);
+    }
+    T ph[KP];
+#pragma unroll
+    for (int q = 0; q < KP; q += VW) lds16(ph + q, s.phi + k * KP + q);
+    const T* cyr = s.cy + k * p.cy_stride + pd.cy_off;
     T w[CPL];
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
@@ -63,31 +124,33 @@ __device__ __forceinline__ void fwd_path(const UvuFwdParams<T>& p, const PathD& 
 #pragma unroll
       for (int q = 1; q < KP; ++q) w[c] = fma(ph[q], a[q][c], w[c]);
     }
+    T cyv[VW];
     if constexpr (D1 <= D3) {
       // fold w into the inputs, then accumulate straight into acc
 #pragma unroll
       for (int m = 0; m < D1; ++m)
 #pragma unroll
         for (int c = 0; c < CPL; ++c) xv[m][c] *= w[c];
-      static_for<CGp::npair>([&](auto P) {
-        constexpr Pair pr = CGp::pair[decltype(P)::value];
-        const T cy = pair_coef<T, CGp, decltype(P)::value>(y);
+      static_for<NP>([&](auto P) {
+        constexpr int Pi = decltype(P)::value;
+        constexpr Pair pr = CGp::pair[Pi];
+        if constexpr (Pi % VW == 0) lds16(cyv, cyr + Pi);
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) acc[pr.m3][c] = fma(cy, xv[pr.m1][c], acc[pr.m3][c]);
+        for (int c = 0; c < CPL; ++c) acc[pr.m3][c] = fma(cyv[Pi % VW], xv[pr.m1][c], acc[pr.m3][c]);
       });
     } else {
       // contract first, then weight the (fewer) output components
       T t[D3][CPL];
-      static_for<CGp::npair>([&](auto P) {
+      static_for<NP>([&](auto P) {
         constexpr int Pi = decltype(P)::value;
         constexpr Pair pr = CGp::pair[Pi];
-        const T cy = pair_coef<T, CGp, Pi>(y);
+        if constexpr (Pi % VW == 0) lds16(cyv, cyr + Pi);
 #pragma unroll
         for (int c = 0; c < CPL; ++c) {
           if constexpr (first_m3<CGp>(Pi))
-            t[pr.m3][c] = cy * xv[pr.m1][c];
+            t[pr.m3][c] = cyv[Pi % VW] * xv[pr.m1][c];
           else
-            t[pr.m3][c] = fma(cy, xv[pr.m1][c], t[pr.m3][c]);
+            t[pr.m3][c] = fma(cyv[Pi % VW], xv[pr.m1][c], t[pr.m3][c]);
         }
       });
       static_for<D3>([&](auto M) {
@@ -98,11 +161,20 @@ __device__ __forceinline__ void fwd_path(const UvuFwdParams<T>& p, const PathD& 
         }
       });
     }
+    if constexpr (kPrefetch) {
+      if (k + 1 < n) {
+#pragma unroll
+        for (int m = 0; m < D1; ++m)
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) xv[m][c] = xn[m][c];
+      }
+    }
   }
 }
 
-template <typename T, int KP, int CPL, int L3>
-__device__ __forceinline__ void fwd_tile(const UvuFwdParams<T>& p, const TileD& tl, int i, int lane) {
+template <typename T, int KP, int CPL, int L1M, int L2M, int L3>
+__device__ __forceinline__ void fwd_tile(const UvuFwdParams<T>& p, const TileD& tl, int i, int lane,
+                                         const FwdSmem<T>& s) {
   constexpr int D3 = 2 * L3 + 1;
   T acc[D3][CPL];
 #pragma unroll
@@ -117,11 +189,40 @@ __device__ __forceinline__ void fwd_tile(const UvuFwdParams<T>& p, const TileD& 
     raise_error(p.err, kErrCsr);
     e1 = e0;
   }
-  for (int pi = tl.pbeg; pi < tl.pend; ++pi) {
-    const PathD& pd = p.paths[pi];
-    dispatch_l1l2<L3>(pd.l1, pd.l2, [&](auto A1, auto A2) {
-      fwd_path<T, KP, CPL, decltype(A1)::value, decltype(A2)::value, L3>(p, pd, chl, e0, e1, acc);
-    });
+  for (int c0 = e0; c0 < e1; c0 += p.chunk) {
+    const int n = min(p.chunk, e1 - c0);
+    // ---- stage: lane k owns edge c0 + k
+    if (lane < n) {
+      const int e = c0 + lane;
+      int j = ldg(p.senders + e);
+      if ((unsigned)j >= (unsigned)p.N) {
+        atomicOr(p.err, kErrIndex);
+        j = -1;
+      }
+      s.j[lane] = j;
+      T ph[KP];
+      load_phi<KP>(ph, p.phi + (size_t)e * p.K, p.K);
+#pragma unroll
+      for (int q = 0; q < KP; ++q) s.phi[lane * KP + q] = j < 0 ? T(0) : ph[q];
+      const T* yrow = p.Y + (size_t)e * p.dim_y;
+      T* cyrow = s.cy + lane * p.cy_stride;
+      for (int pi = tl.pbeg; pi < tl.pend; ++pi) {
+        const PathD& pd = p.paths[pi];
+        dispatch_l1l2<L3, L1M, L2M>(pd.l1, pd.l2, [&](auto A1, auto A2) {
+          stage_cy<T, decltype(A1)::value, decltype(A2)::value, L3>(yrow, cyrow + pd.cy_off);
+        });
+      }
+      if (j < 0) s.j[lane] = 0;  // a skipped edge contributes zero (phi = 0)
+    }
+    __syncwarp();
+    // ---- sweep: every path of the tile over the staged chunk
+    for (int pi = tl.pbeg; pi < tl.pend; ++pi) {
+      const PathD& pd = p.paths[pi];
+      dispatch_l1l2<L3, L1M, L2M>(pd.l1, pd.l2, [&](auto A1, auto A2) {
+        fwd_path<T, KP, CPL, decltype(A1)::value, decltype(A2)::value, L3>(p, pd, s, n, chl, acc);
+      });
+    }
+    __syncwarp();
   }
   if (active) {
     T* o = p.out + (size_t)i * p.c_out + tl.off + chl;
@@ -130,48 +231,82 @@ __device__ __forceinline__ void fwd_tile(const UvuFwdParams<T>& p, const TileD& 
   }
 }
 
-template <typename T, int KP, int CPL>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+// fp32: two CTAs per SM (register cap 128) measured faster than one CTA with
+// more registers; fp64 spills under that cap, so it keeps one.
+template <typename T, int KP, int CPL, int L1M, int L2M, int L3M>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, sizeof(T) == 4 ? 2 : 1)
 uvu_fwd_kernel(const __grid_constant__ UvuFwdParams<T> p) {
-  const int lane = threadIdx.x & 31;
-  const long long task = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
-  if (task >= (long long)p.N * p.n_tiles) return;
-  const int i = (int)(task / p.n_tiles);
-  const TileD& tl = p.tiles[(int)(task % p.n_tiles)];
-  dispatch_l(tl.l, [&](auto L) { fwd_tile<T, KP, CPL, decltype(L)::value>(p, tl, i, lane); });
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long long task = (long long)blockIdx.x * kWarpsPerBlock + warp;
+  const long long per_win = (long long)kWin * p.n_tiles;
+  const long long win = task / per_win;
+  const int r = (int)(task - win * per_win);
+  const int tile = r / kWin;
+  const long long i = win * kWin + (r % kWin);
+  if (i >= p.N) return;
+  const TileD& tl = p.tiles[tile];
+  const FwdSmem<T> s = fwd_smem<T, KP>(p, warp);
+  dispatch_l<L3M>(tl.l, [&](auto L) {
+    fwd_tile<T, KP, CPL, L1M, L2M, decltype(L)::value>(p, tl, (int)i, lane, s);
+  });
 }
 
 }  // namespace
 
-template <typename T, int KP, int CPL>
+template <typename T, int KP, int CPL, int L1M, int L2M, int L3M>
 cudaError_t launch_uvu_fwd(const UvuFwdParams<T>& p, cudaStream_t s) {
-  const long long tasks = (long long)p.N * p.n_tiles;
+  const long long wins = ((long long)p.N + kWin - 1) / kWin;
+  const long long tasks = wins * kWin * p.n_tiles;
   if (tasks == 0) return cudaSuccess;
   const long long blocks = (tasks + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  uvu_fwd_kernel<T, KP, CPL><<<(unsigned)blocks, kWarpsPerBlock * 32, 0, s>>>(p);
+  const size_t smem = (size_t)p.warp_smem * kWarpsPerBlock;
+  auto kern = uvu_fwd_kernel<T, KP, CPL, L1M, L2M, L3M>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<(unsigned)blocks, kWarpsPerBlock * 32, smem, s>>>(p);
   return cudaGetLastError();
 }
 
-#define TPC_INST(T, KP, CPL) \
-  template cudaError_t launch_uvu_fwd<T, KP, CPL>(const UvuFwdParams<T>&, cudaStream_t);
+// degree profiles (max input l, max SH l, max output l): see plan.cpp
+#define TPC_INST(T, KP, CPL, A, B, C) \
+  template cudaError_t launch_uvu_fwd<T, KP, CPL, A, B, C>(const UvuFwdParams<T>&, cudaStream_t);
+#define TPC_INST_P(T, KP, CPL) \
+  TPC_INST(T, KP, CPL, 2, 2, 2) TPC_INST(T, KP, CPL, 1, 3, 3) TPC_INST(T, KP, CPL, 3, 3, 3)
 #if TPC_WANT(0)
-TPC_INST(float, 8, 1)
+TPC_INST_P(float, 8, 1)
+TPC_INST(float, 8, 1, 4, 4, 4)
 #endif
 #if TPC_WANT(1)
-TPC_INST(float, 8, 2)
+TPC_INST_P(float, 8, 2)
 #endif
 #if TPC_WANT(2)
-TPC_INST(float, 16, 1)
+TPC_INST(float, 8, 2, 4, 4, 4)
 #endif
 #if TPC_WANT(3)
-TPC_INST(float, 16, 2)
+TPC_INST_P(float, 16, 1)
+TPC_INST(float, 16, 1, 4, 4, 4)
 #endif
 #if TPC_WANT(4)
-TPC_INST(double, 8, 1)
+TPC_INST_P(float, 16, 2)
+TPC_INST(float, 16, 2, 4, 4, 4)
 #endif
 #if TPC_WANT(5)
-TPC_INST(double, 16, 1)
+TPC_INST_P(double, 8, 1)
+TPC_INST(double, 8, 1, 4, 4, 4)
 #endif
+#if TPC_WANT(6)
+TPC_INST_P(double, 8, 2)
+#endif
+#if TPC_WANT(7)
+TPC_INST_P(double, 16, 1)
+TPC_INST(double, 16, 1, 4, 4, 4)
+#endif
+#if TPC_WANT(8)
+TPC_INST_P(double, 16, 2)
+#endif
+#undef TPC_INST_P
 #undef TPC_INST
 
 }  // namespace tpc
