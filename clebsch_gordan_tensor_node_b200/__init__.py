@@ -13,7 +13,7 @@ from typing import Optional, Tuple
 from ._lib import (TP_F32, TP_F64, TP_UVU, TP_UVW, PathInfo, PlanInfo, TpConvError, check, lib)
 
 __all__ = ["Plan", "tp_conv_plan", "tp_csr_build", "tp_csr_transpose", "tp_conv_forward",
-           "tp_conv_backward", "tp_get_device_error", "TpConvError"]
+           "tp_conv_backward", "tp_conv_backward_noalloc", "tp_get_device_error", "TpConvError"]
 
 
 def _torch():
@@ -192,6 +192,28 @@ def tp_conv_backward(plan: Plan, x, Y, phi, A, rowptr, senders, colptr, srcedge,
                                  _ptr(senders), _ptr(colptr), _ptr(srcedge), _ptr(srcrecv),
                                  _ptr(grad_out), N, E, _ptr(gx), _ptr(gY), _ptr(gphi), _ptr(gA),
                                  _ptr(ws), wsb, _stream(stream)), "tp_conv_backward")
+    return gx, gY, gphi, gA
+
+
+def tp_conv_backward_noalloc(plan: Plan, x, Y, phi, A, rowptr, senders, colptr, srcedge, srcrecv,
+                             grad_out, out=None, stream=None):
+    """tp_conv_backward without a workspace argument: the library's static
+    device scratch holds the grad_A partials (see include/tpconv.h). The output
+    tensors are the caller's; pass `out` to avoid any allocation here too."""
+    torch = _torch()
+    N, E = x.shape[0], senders.numel()
+    dt = plan.torch_dtype
+    _need(grad_out, dt, (N, plan.c_out), "grad_out")
+    if out is None:
+        out = (torch.empty(N, plan.c_in, dtype=dt, device=x.device),
+               torch.empty(E, plan.dim_y, dtype=dt, device=x.device),
+               torch.empty(E, plan.n_radial, dtype=dt, device=x.device),
+               torch.empty(plan.n_radial, plan.n_w, dtype=dt, device=x.device))
+    gx, gY, gphi, gA = out
+    check(lib().tp_conv_backward_noalloc(plan.handle, _ptr(x), _ptr(Y), _ptr(phi), _ptr(A), _ptr(rowptr),
+                                         _ptr(senders), _ptr(colptr), _ptr(srcedge), _ptr(srcrecv),
+                                         _ptr(grad_out), N, E, _ptr(gx), _ptr(gY), _ptr(gphi), _ptr(gA),
+                                         _stream(stream)), "tp_conv_backward_noalloc")
     return gx, gY, gphi, gA
 
 

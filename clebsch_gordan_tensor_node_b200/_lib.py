@@ -50,6 +50,9 @@ SIGNATURES = {
     "tp_conv_backward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_void_p,
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "tp_conv_backward_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                         c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_void_p,
+                                         c_void_p, c_void_p, c_void_p, c_void_p]),
     "tp_get_device_error": (c_int, [c_void_p]),
     "tp_status_string": (c_char_p, [c_int]),
     "tp_last_error_message": (c_char_p, []),

@@ -29,6 +29,7 @@ UNITS = {
     "uvu_bwd.cu": 6,
     "csr.cu": 1,
     "api.cu": 1,
+    "noalloc.cu": 1,
     "plan.cpp": 1,
     "cg_host.cpp": 1,
 }

@@ -160,6 +160,11 @@ int backward_uvu(const Plan& P, const void* x, const void* Y, const void* phi, c
 }
 
 }  // namespace
+
+// Shared with other translation units of the library.
+int set_error_message(int status, const std::string& m) { return fail(status, m); }
+int device_error_word(int** out) { return error_word(out); }
+
 }  // namespace tpc
 
 using namespace tpc;

@@ -33,3 +33,12 @@ cudaError_t csr_transpose(int N, int E, const int* rowptr, const int* senders, i
 #define TPC_SET -1
 #endif
 #define TPC_WANT(k) (TPC_SET < 0 || TPC_SET == (k))
+
+#include <string>
+
+namespace tpc {
+// Record a host-side failure for tp_last_error_message; returns status.
+int set_error_message(int status, const std::string& msg);
+// Device address of the current device's error word.
+int device_error_word(int** out);
+}  // namespace tpc

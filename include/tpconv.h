@@ -182,6 +182,30 @@ int tp_conv_backward(tp_plan_t plan, const void* x, const void* Y, const void* p
                      int64_t n_nodes, int64_t n_edges, void* grad_x, void* grad_Y, void* grad_phi,
                      void* grad_A, void* ws, size_t ws_bytes, void* stream);
 
+/* tp_conv_backward for callers that cannot allocate device memory (no
+ * counterpart in the pages: it is a service of this library). Plugins run from
+ * another engine's execution step, code running while a stream capture is
+ * open, or processes held to a fixed memory reservation may be unable to
+ * cudaMalloc the workspace tp_conv_backward asks for. This entry point takes
+ * the same arguments minus the workspace and allocates nothing: the grad_A
+ * partial sums live in a static 16 MiB array of device memory inside the
+ * library, which every GPU that loads the library keeps reserved until the
+ * process exits. Limits: channelwise (uvu) plans only (else TP_EUNSUPPORTED);
+ * one slot of partials takes K * N_w * scalar-size bytes and must fit in the
+ * 16 MiB (else TP_EWORKSPACE with the sizes in tp_last_error_message); with
+ * fewer slots than tp_conv_backward uses, results differ from it only by the
+ * order of the grad_A additions. The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current: make
+ * that first call before any stream capture. Every call on a device shares the
+ * one array and leaves its contents behind (each call clears what it needs
+ * first); calls that may overlap on the GPU -- different streams, or threads
+ * without ordering -- race on it and give wrong results. */
+int tp_conv_backward_noalloc(tp_plan_t plan, const void* x, const void* Y, const void* phi,
+                             const void* A, const int32_t* rowptr, const int32_t* senders,
+                             const int32_t* colptr, const int32_t* srcedge, const int32_t* srcrecv,
+                             const void* grad_out, int64_t n_nodes, int64_t n_edges, void* grad_x,
+                             void* grad_Y, void* grad_phi, void* grad_A, void* stream);
+
 /* Synchronise `stream`, then read and clear the device error word of the
  * current device. Returns TP_OK, TP_EDEVICE_INDEX, TP_EDEVICE_CSR or
  * TP_ECUDA. */
