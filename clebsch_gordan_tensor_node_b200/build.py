@@ -27,6 +27,8 @@ CG_LMAX = 6
 UNITS = {
     "uvu_fwd.cu": 9,
     "uvu_bwd.cu": 6,
+    "uvw.cu": 4,
+    "gemm.cu": 1,
     "csr.cu": 1,
     "api.cu": 1,
     "noalloc.cu": 1,

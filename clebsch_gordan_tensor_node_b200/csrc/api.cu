@@ -159,6 +159,183 @@ int backward_uvu(const Plan& P, const void* x, const void* Y, const void* phi, c
   return e == cudaSuccess ? TP_OK : cuda_fail(e, "grad_A reduction launch");
 }
 
+// ---------------------------------------------------------------- uvw
+
+template <typename T>
+cudaError_t sbuild(const Plan& P, const UvwSParams<T>& p, int dir, cudaStream_t s) {
+  return P.KP == 8 ? launch_uvw_sbuild<T, 8>(p, dir, s) : launch_uvw_sbuild<T, 16>(p, dir, s);
+}
+
+template <typename T>
+void fill_blocks(UvwSParams<T>& p, const std::vector<UvwBlockD>& blocks, const std::vector<PathD>& paths) {
+  std::memset(p.blocks, 0, sizeof(p.blocks));
+  std::memset(p.paths, 0, sizeof(p.paths));
+  std::memcpy(p.blocks, blocks.data(), blocks.size() * sizeof(UvwBlockD));
+  std::memcpy(p.paths, paths.data(), paths.size() * sizeof(PathD));
+  p.n_blocks = (int)blocks.size();
+}
+
+size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+// m_g = S_g B_g for every output block of one receiver chunk (rows -> out).
+template <typename T>
+cudaError_t mix_out(const Plan& P, const T* S, const T* Bf, T* out, int r0, int nr, int nr_alloc,
+                    const std::vector<UvwBlockD>& blocks, const std::vector<long long>& b_off, long long ld_out,
+                    cudaStream_t s) {
+  GemmBatch<T> gb;
+  int n = 0, mm = 0, mn = 0;
+  for (size_t g = 0; g < blocks.size(); ++g) {
+    const UvwBlockD& b = blocks[g];
+    GemmProb<T>& q = gb.prob[n++];
+    const int dc = 2 * b.l + 1;
+    q.X = S + (size_t)nr_alloc * b.s_off;
+    q.B = Bf + b_off[g];
+    q.G = nullptr;
+    q.C = out;
+    q.c = RowBlocked{r0, dc, ld_out, b.out_off, b.mul_own};
+    q.M = nr * dc; q.N = b.mul_own; q.D = b.dcols; q.accumulate = 0;
+    mm = std::max(mm, q.M);
+    mn = std::max(mn, q.N);
+    if (n == kMaxGemmBatch || g + 1 == blocks.size()) {
+      cudaError_t e = launch_gemm<T>(0, gb, n, mm, mn, s);
+      if (e != cudaSuccess) return e;
+      n = mm = mn = 0;
+    }
+  }
+  return cudaSuccess;
+}
+
+template <typename T>
+int forward_uvw(const Plan& P, const void* x, const void* Y, const void* phi, const void* A, const int* rowptr,
+                const int* senders, int N, int E, void* out, void* ws, int* err, cudaStream_t s) {
+  const size_t b = sizeof(T);
+  T* Bf = (T*)ws;
+  T* S = (T*)((char*)ws + align256((size_t)P.K * P.n_w * b));
+  cudaError_t e = launch_pack_a<T>(P.pack, (const T*)A, Bf, nullptr, s);
+  if (e != cudaSuccess) return cuda_fail(e, "pack A");
+  std::vector<long long> bf_off;
+  {
+    long long off = 0;
+    for (auto& g : P.uvw_out) {
+      bf_off.push_back(off);
+      off += (long long)g.dcols * g.mul_own;
+    }
+  }
+  UvwSParams<T> sp;
+  sp.feat = (const T*)x; sp.Y = (const T*)Y; sp.phi = (const T*)phi;
+  sp.ptr = rowptr; sp.nbr = senders; sp.eid = nullptr; sp.S = S; sp.err = err;
+  sp.N = N; sp.E = E; sp.K = P.K; sp.ld_feat = P.c_in; sp.dim_y = P.dim_y; sp.n_feat_rows = N;
+  fill_blocks(sp, P.uvw_out, P.paths_fwd);
+  const int NR = uvw_chunk_rows(P, N, 0);
+  sp.nr_alloc = NR;
+  for (int r0 = 0; r0 < N; r0 += NR) {
+    sp.r0 = r0;
+    sp.nr = std::min(NR, N - r0);
+    if ((e = sbuild<T>(P, sp, 0, s)) != cudaSuccess) return cuda_fail(e, "uvw state build");
+    if ((e = mix_out<T>(P, S, Bf, (T*)out, r0, sp.nr, NR, P.uvw_out, bf_off, P.c_out, s)) != cudaSuccess)
+      return cuda_fail(e, "uvw mixing");
+  }
+  return TP_OK;
+}
+
+template <typename T>
+int backward_uvw(const Plan& P, const void* x, const void* Y, const void* phi, const void* A, const int* rowptr,
+                 const int* senders, const int* colptr, const int* srcedge, const int* srcrecv, const void* gout,
+                 int N, int E, void* gx, void* gY, void* gphi, void* gA, void* ws, int* err, cudaStream_t s) {
+  const size_t b = sizeof(T);
+  const size_t a = align256((size_t)P.K * P.n_w * b);
+  T* Bf = (T*)ws;
+  T* Ba = (T*)((char*)ws + a);
+  T* Ab = (T*)((char*)ws + 2 * a);
+  const int NR = uvw_chunk_rows(P, N, 0), NS = uvw_chunk_rows(P, N, 1);
+  const size_t s0 = align256((size_t)NR * P.s_row_elems * b), s1 = align256((size_t)NS * P.sa_row_elems * b);
+  T* S = (T*)((char*)ws + 3 * a);
+  T* Sb = (T*)((char*)ws + 3 * a + std::max(s0, s1));
+  cudaError_t e = launch_pack_a<T>(P.pack, (const T*)A, Bf, Ba, s);
+  if (e != cudaSuccess) return cuda_fail(e, "pack A");
+  std::vector<long long> bf_off, ba_off;
+  {
+    long long off = 0;
+    for (auto& g : P.uvw_out) {
+      bf_off.push_back(off);
+      off += (long long)g.dcols * g.mul_own;
+    }
+    off = 0;
+    for (auto& g : P.uvw_in) {
+      ba_off.push_back(off);
+      off += (long long)g.dcols * g.mul_own;
+    }
+  }
+  // ---- receiver chunks: S, A_bar += S^T m_bar, S_bar = m_bar B^T, edge pass
+  UvwSParams<T> sp;
+  sp.feat = (const T*)x; sp.Y = (const T*)Y; sp.phi = (const T*)phi;
+  sp.ptr = rowptr; sp.nbr = senders; sp.eid = nullptr; sp.S = S; sp.err = err;
+  sp.N = N; sp.E = E; sp.K = P.K; sp.ld_feat = P.c_in; sp.dim_y = P.dim_y; sp.n_feat_rows = N;
+  sp.nr_alloc = NR;
+  fill_blocks(sp, P.uvw_out, P.paths_fwd);
+  UvwEdgeParams<T> ep;
+  ep.x = (const T*)x; ep.Y = (const T*)Y; ep.phi = (const T*)phi; ep.Sbar = Sb;
+  ep.rowptr = rowptr; ep.senders = senders; ep.gY = (T*)gY; ep.gphi = (T*)gphi; ep.err = err;
+  ep.N = N; ep.E = E; ep.K = P.K; ep.c_in = P.c_in; ep.dim_y = P.dim_y; ep.nr_alloc = NR;
+  std::memset(ep.blocks, 0, sizeof(ep.blocks));
+  std::memset(ep.paths, 0, sizeof(ep.paths));
+  std::memcpy(ep.blocks, P.uvw_out.data(), P.uvw_out.size() * sizeof(UvwBlockD));
+  std::memcpy(ep.paths, P.paths_fwd.data(), P.paths_fwd.size() * sizeof(PathD));
+  ep.n_blocks = (int)P.uvw_out.size();
+  for (int r0 = 0; r0 < N; r0 += NR) {
+    const int nr = std::min(NR, N - r0);
+    sp.r0 = r0;
+    sp.nr = nr;
+    if ((e = sbuild<T>(P, sp, 0, s)) != cudaSuccess) return cuda_fail(e, "uvw state build");
+    for (int pass = 0; pass < 2; ++pass) {
+      GemmBatch<T> gb;
+      int n = 0, mm = 0, mn = 0;
+      for (size_t g = 0; g < P.uvw_out.size(); ++g) {
+        const UvwBlockD& bd = P.uvw_out[g];
+        const int dc = 2 * bd.l + 1;
+        GemmProb<T>& q = gb.prob[n++];
+        q.G = (const T*)gout;
+        q.g = RowBlocked{r0, dc, P.c_out, bd.out_off, bd.mul_own};
+        q.M = nr * dc; q.N = bd.mul_own; q.D = bd.dcols;
+        if (pass == 0) {            // A_bar_g (+)= S_g^T m_bar_g
+          q.X = S + (size_t)NR * bd.s_off; q.B = nullptr; q.C = Ab + bf_off[g];
+          q.accumulate = r0 > 0;
+          mm = std::max(mm, q.D); mn = std::max(mn, q.N);
+        } else {                    // S_bar_g = m_bar_g B_g^T
+          q.X = nullptr; q.B = Bf + bf_off[g]; q.C = Sb + (size_t)NR * bd.s_off;
+          q.accumulate = 0;
+          mm = std::max(mm, q.M); mn = std::max(mn, q.D);
+        }
+        if (n == kMaxGemmBatch || g + 1 == P.uvw_out.size()) {
+          if ((e = launch_gemm<T>(pass == 0 ? 2 : 1, gb, n, mm, mn, s)) != cudaSuccess)
+            return cuda_fail(e, "uvw backward GEMM");
+          n = mm = mn = 0;
+        }
+      }
+    }
+    ep.r0 = r0;
+    ep.nr = nr;
+    e = P.KP == 8 ? launch_uvw_edge<T, 8>(ep, s) : launch_uvw_edge<T, 16>(ep, s);
+    if (e != cudaSuccess) return cuda_fail(e, "uvw edge pass");
+  }
+  // ---- source chunks: S' over the source view, x_bar = S' B'
+  UvwSParams<T> ap;
+  ap.feat = (const T*)gout; ap.Y = (const T*)Y; ap.phi = (const T*)phi;
+  ap.ptr = colptr; ap.nbr = srcrecv; ap.eid = srcedge; ap.S = S; ap.err = err;
+  ap.N = N; ap.E = E; ap.K = P.K; ap.ld_feat = P.c_out; ap.dim_y = P.dim_y; ap.n_feat_rows = N;
+  ap.nr_alloc = NS;
+  fill_blocks(ap, P.uvw_in, P.paths_adj);
+  for (int s0r = 0; s0r < N; s0r += NS) {
+    ap.r0 = s0r;
+    ap.nr = std::min(NS, N - s0r);
+    if ((e = sbuild<T>(P, ap, 1, s)) != cudaSuccess) return cuda_fail(e, "uvw source state build");
+    if ((e = mix_out<T>(P, S, Ba, (T*)gx, s0r, ap.nr, NS, P.uvw_in, ba_off, P.c_in, s)) != cudaSuccess)
+      return cuda_fail(e, "uvw grad_x mixing");
+  }
+  e = launch_unpack_a<T>(P.pack, Ab, (T*)gA, s);
+  return e == cudaSuccess ? TP_OK : cuda_fail(e, "unpack grad_A");
+}
+
 }  // namespace
 
 // Shared with other translation units of the library.
@@ -298,7 +475,12 @@ int tp_conv_forward(tp_plan_t plan, const void* x, const void* Y, const void* ph
   int* err = nullptr;
   if ((st = error_word(&err))) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  if (P.mode != TP_UVU) return fail(TP_EUNSUPPORTED, "uvw forward is not built yet");
+  if (P.mode == TP_UVW) {
+    if (!ws) return fail(TP_EWORKSPACE, "uvw forward needs a workspace");
+    return P.dtype == TP_F32
+               ? forward_uvw<float>(P, x, Y, phi, A, rowptr, senders, (int)n_nodes, (int)n_edges, out, ws, err, s)
+               : forward_uvw<double>(P, x, Y, phi, A, rowptr, senders, (int)n_nodes, (int)n_edges, out, ws, err, s);
+  }
   return P.dtype == TP_F32
              ? forward_uvu<float>(P, x, Y, phi, A, rowptr, senders, (int)n_nodes, (int)n_edges, out, err, s)
              : forward_uvu<double>(P, x, Y, phi, A, rowptr, senders, (int)n_nodes, (int)n_edges, out, err, s);
@@ -326,11 +508,16 @@ int tp_conv_backward(tp_plan_t plan, const void* x, const void* Y, const void* p
   int* err = nullptr;
   if ((st = error_word(&err))) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  if (P.mode != TP_UVU) return fail(TP_EUNSUPPORTED, "uvw backward is not built yet");
   if (n_nodes == 0) {
     cudaError_t e = cudaMemsetAsync(grad_A, 0, (size_t)P.K * P.n_w * (P.dtype == TP_F32 ? 4 : 8), s);
     return e == cudaSuccess ? TP_OK : cuda_fail(e, "memset grad_A");
   }
+  if (P.mode == TP_UVW)
+    return P.dtype == TP_F32
+               ? backward_uvw<float>(P, x, Y, phi, A, rowptr, senders, colptr, srcedge, srcrecv, grad_out,
+                                     (int)n_nodes, (int)n_edges, grad_x, grad_Y, grad_phi, grad_A, ws, err, s)
+               : backward_uvw<double>(P, x, Y, phi, A, rowptr, senders, colptr, srcedge, srcrecv, grad_out,
+                                      (int)n_nodes, (int)n_edges, grad_x, grad_Y, grad_phi, grad_A, ws, err, s);
   return P.dtype == TP_F32
              ? backward_uvu<float>(P, x, Y, phi, A, rowptr, senders, colptr, srcedge, srcrecv, grad_out,
                                    (int)n_nodes, (int)n_edges, grad_x, grad_Y, grad_phi, grad_A, ws, err, s)

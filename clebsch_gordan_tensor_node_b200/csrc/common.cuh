@@ -32,6 +32,7 @@ struct PathD {          // one coupling path (l1, l2) -> l3
   int mul_in;
   int mul_out;
   int cy_off;           // forward: first cY slot of the path in a staged edge row
+  int col_off;          // uvw: first column of the path in its owner block's state row
 };
 
 struct TileD {          // one channel tile of one irrep block
@@ -79,6 +80,71 @@ struct UvuSrcParams {         // backward: source-owned grad_x, grad_A partials
   int n_tiles, n_slots;
   TileD tiles[kMaxTiles];     // one per (input block, channel tile)
   PathD paths[kMaxPaths];     // grouped by input block
+};
+
+// ---- fully connected (uvw) path
+
+constexpr int kMaxBlocks = 32;
+
+struct UvwBlockD {      // owner block of a receiver-state (S) or source-state (S') build
+  int l;                // degree of the owner block
+  int pbeg, pend;       // its paths in the kernel's path array
+  int dcols;            // state columns per owner row: sum over paths of K * gathered mul
+  long long s_off;      // region of the block in a state chunk, in units of chunk rows
+  int out_off;          // owner block offset in the owner's row (out or grad_x)
+  int mul_own;          // multiplicity of the owner block
+};
+
+template <typename T>
+struct UvwSParams {           // S (dir 0: receivers gather x) or S' (dir 1: sources gather grad_out)
+  const T* feat; const T* Y; const T* phi;
+  const int* ptr; const int* nbr; const int* eid;   // eid = NULL: edge id = position
+  T* S; int* err;
+  int N, E, K, ld_feat, dim_y, n_feat_rows;
+  int r0, nr, nr_alloc, n_blocks;
+  UvwBlockD blocks[kMaxBlocks];
+  PathD paths[kMaxPaths];     // x_off / mul_in describe the gathered block
+};
+
+template <typename T>
+struct UvwEdgeParams {        // backward: edge-owned grad_phi, grad_Y from S_bar
+  const T* x; const T* Y; const T* phi; const T* Sbar;
+  const int* rowptr; const int* senders;
+  T* gY; T* gphi; int* err;
+  int N, E, K, c_in, dim_y;
+  int r0, nr, nr_alloc, n_blocks;
+  UvwBlockD blocks[kMaxBlocks];
+  PathD paths[kMaxPaths];
+};
+
+struct PackPath {       // where the A columns of one path go in the packed GEMM operands
+  int w_off, mi, mo, colf, cola;
+  long long bf_off, ba_off;
+};
+
+struct UvwPackParams {
+  int K, n_w, n_paths;
+  PackPath paths[kMaxPaths];
+};
+
+struct RowBlocked {     // row m = (owner r, component c) -> (r0 + r) * ld_outer + off + c * n
+  int r0, dcomp;
+  long long ld_outer;
+  int off, n;
+};
+
+template <typename T>
+struct GemmProb {
+  const T* X; const T* B; const T* G; T* C;
+  RowBlocked g, c;
+  int M, N, D, accumulate;
+};
+
+constexpr int kMaxGemmBatch = 16;
+
+template <typename T>
+struct GemmBatch {
+  GemmProb<T> prob[kMaxGemmBatch];
 };
 
 // ------------------------------------------------------------------ compile-time helpers

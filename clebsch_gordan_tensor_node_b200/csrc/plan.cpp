@@ -240,7 +240,95 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
   P.fwd_chunk = std::max(1, std::min(32, (20 * 1024) / (P.cy_stride * bsz)));
   P.fwd_warp_smem = 32 * 4 + 32 * P.KP * bsz + P.fwd_chunk * P.cy_stride * bsz;
   P.fwd_warp_smem = (P.fwd_warp_smem + 15) / 16 * 16;
+  if (mode == TP_UVW) {
+    if ((int)P.bout.size() > kMaxBlocks || (int)P.bin.size() > kMaxBlocks) {
+      msg = "more than " + std::to_string(kMaxBlocks) + " irrep blocks";
+      return TP_EUNSUPPORTED;
+    }
+    // receiver state S (Sobek §4.2): per output block g, rows (receiver, m3),
+    // columns (path of g, q, u); the mixing operand B_g packs A's rows in the
+    // same (path, q, u) order
+    long long s_off = 0, bf_off = 0;
+    P.pack.K = P.K;
+    P.pack.n_w = (int)P.n_w;
+    P.pack.n_paths = (int)P.paths.size();
+    for (size_t g = 0; g < P.bout.size(); ++g) {
+      UvwBlockD b{};
+      b.l = P.bout[g].l;
+      b.pbeg = (int)P.paths_fwd.size();
+      int cols = 0;
+      for (int pi : by_out[g]) {
+        const HostPath& h = P.paths[pi];
+        PathD d{};
+        d.l1 = (int8_t)h.l1; d.l2 = (int8_t)h.l2; d.l3 = (int8_t)h.l3;
+        d.x_off = h.x_off; d.mul_in = h.mul_in; d.out_off = h.out_off; d.mul_out = h.mul_out;
+        d.w_off = (int)h.w_off;
+        d.col_off = cols;
+        P.pack.paths[pi].w_off = (int)h.w_off;
+        P.pack.paths[pi].mi = h.mul_in;
+        P.pack.paths[pi].mo = h.mul_out;
+        P.pack.paths[pi].colf = cols;
+        P.pack.paths[pi].bf_off = bf_off;
+        cols += P.K * h.mul_in;
+        P.paths_fwd.push_back(d);
+      }
+      b.pend = (int)P.paths_fwd.size();
+      b.dcols = cols;
+      b.s_off = s_off;
+      b.out_off = P.bout[g].offset;
+      b.mul_own = P.bout[g].mul;
+      s_off += (long long)(2 * b.l + 1) * cols;
+      bf_off += (long long)cols * P.bout[g].mul;
+      P.uvw_out.push_back(b);
+    }
+    P.s_row_elems = s_off;
+    // source state S' for x_bar: per input block b, rows (source, m1), columns
+    // (path from b, q, w); B'_b packs A's rows in (path, q, w) order
+    long long sa_off = 0, ba_off = 0;
+    for (size_t b1 = 0; b1 < P.bin.size(); ++b1) {
+      UvwBlockD b{};
+      b.l = P.bin[b1].l;
+      b.pbeg = (int)P.paths_adj.size();
+      int cols = 0;
+      for (int pi : by_in[b1]) {
+        const HostPath& h = P.paths[pi];
+        PathD d{};
+        d.l1 = (int8_t)h.l1; d.l2 = (int8_t)h.l2; d.l3 = (int8_t)h.l3;
+        d.x_off = h.out_off;            // gathered: the grad_out block of the path
+        d.mul_in = h.mul_out;
+        d.out_off = h.x_off; d.mul_out = h.mul_in;
+        d.w_off = (int)h.w_off;
+        d.col_off = cols;
+        P.pack.paths[pi].cola = cols;
+        P.pack.paths[pi].ba_off = ba_off;
+        cols += P.K * h.mul_out;
+        P.paths_adj.push_back(d);
+      }
+      b.pend = (int)P.paths_adj.size();
+      b.dcols = cols;
+      b.s_off = sa_off;
+      b.out_off = P.bin[b1].offset;
+      b.mul_own = P.bin[b1].mul;
+      sa_off += (long long)(2 * b.l + 1) * cols;
+      ba_off += (long long)cols * P.bin[b1].mul;
+      P.uvw_in.push_back(b);
+    }
+    P.sa_row_elems = sa_off;
+    const size_t bsz2 = dtype == TP_F32 ? 4 : 8;
+    if ((size_t)std::max(P.s_row_elems, P.sa_row_elems) * bsz2 > kUvwChunkBytes) {
+      msg = "one node's uvw state exceeds the state chunk budget";
+      return TP_EUNSUPPORTED;
+    }
+  }
   return TP_OK;
+}
+
+int uvw_chunk_rows(const Plan& p, long long n_nodes, int dir) {
+  const size_t b = p.dtype == TP_F32 ? 4 : 8;
+  const long long per = std::max<long long>(1, (dir == 0 ? p.s_row_elems : p.sa_row_elems));
+  long long r = (long long)(kUvwChunkBytes / (per * b));
+  r = std::max<long long>(1, std::min<long long>(r, std::max<long long>(1, n_nodes)));
+  return (int)r;
 }
 
 int uvu_src_slots(const Plan& p, long long n_nodes) {
@@ -256,6 +344,14 @@ size_t workspace_bytes(const Plan& p, long long n_nodes, int pass) {
   size_t bytes = 0;
   if (p.mode == TP_UVU) {
     if (pass == 1) bytes = (size_t)uvu_src_slots(p, n_nodes) * p.K * p.n_w * b;
+  } else {
+    // packed A (forward operand; plus adjoint operand and packed A_bar in the
+    // backward), each 256-byte aligned, and one (forward) or two (backward)
+    // state chunks
+    const size_t a = ((size_t)p.K * p.n_w * b + 255) / 256 * 256;
+    const size_t s0 = ((size_t)uvw_chunk_rows(p, n_nodes, 0) * p.s_row_elems * b + 255) / 256 * 256;
+    const size_t s1 = ((size_t)uvw_chunk_rows(p, n_nodes, 1) * p.sa_row_elems * b + 255) / 256 * 256;
+    bytes = pass == 0 ? a + s0 : 3 * a + 2 * std::max(s0, s1);
   }
   return (bytes + 255) / 256 * 256;
 }

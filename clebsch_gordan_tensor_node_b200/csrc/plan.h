@@ -37,7 +37,20 @@ struct Plan {
   std::vector<TileD> in_tiles;    // (input block, channel tile), paths_by_in ranges
   std::vector<PathD> paths_by_in;
   std::vector<PathD> paths_canon;
+  // fully connected (uvw) tables
+  std::vector<UvwBlockD> uvw_out;   // output blocks, with paths_fwd ranges
+  std::vector<PathD> paths_fwd;     // by output block; gathered = x block
+  std::vector<UvwBlockD> uvw_in;    // input blocks, with paths_adj ranges
+  std::vector<PathD> paths_adj;     // by input block; gathered = grad_out block
+  UvwPackParams pack{};
+  long long s_row_elems = 0;        // state elements per receiver (S)
+  long long sa_row_elems = 0;       // state elements per source (S')
 };
+
+// Bytes of one uvw state chunk (the scratch budget of Sobek App. B.2).
+constexpr size_t kUvwChunkBytes = size_t(256) << 20;
+// Owners per uvw state chunk for a problem of n_nodes nodes (dir 0: S, 1: S').
+int uvw_chunk_rows(const Plan& p, long long n_nodes, int dir);
 
 // Returns 0 or a negative tp_status; msg receives a human-readable reason.
 int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_radial, int mode,

@@ -65,8 +65,14 @@ def _blocks(pr: Problem, p: Path, x, Y, src):
     return xj, Ye
 
 
+def _chunk(pr: Problem, chunk: int) -> int:
+    """Edges per materialised chunk, bounded so that W [chunk, N_w] stays <= 1 GiB."""
+    return max(1, min(chunk, (1 << 27) // max(1, pr.n_w)))
+
+
 def forward(pr: Problem, x, Y, phi, A, src, dst, n_nodes: int, chunk: int = 65536):
     """Materialised forward: per edge chunk W = phi A, messages M, scatter-add."""
+    chunk = _chunk(pr, chunk)
     x = np.asarray(x, np.float64)
     out = np.zeros((n_nodes, pr.c_out))
     E = len(src)
@@ -94,6 +100,7 @@ def backward(pr: Problem, x, Y, phi, A, src, dst, grad_out, n_nodes: int, chunk:
 
     Returns grad_x [N, C_x], grad_Y [E, dimY], grad_phi [E, K], grad_A [K, N_w].
     """
+    chunk = _chunk(pr, chunk)
     x = np.asarray(x, np.float64)
     A = np.asarray(A, np.float64)
     g = np.asarray(grad_out, np.float64)

@@ -61,6 +61,8 @@ SPEC = ("8x0e+8x1o+8x2e", 2, "8x0e+8x1o+8x1e+8x2e+8x2o", 8, "uvu")
 def test_empty_graph():
     out = _run_and_compare(SPEC, "f64", 5, [], [])
     assert not out.any()
+    out = _run_and_compare(("2x0e+3x1o", 2, "3x0e+2x1o+2x2e", 3, "uvw"), "f32", 5, [], [])
+    assert not out.any()
 
 
 def test_isolated_and_hub_nodes():
@@ -71,6 +73,7 @@ def test_isolated_and_hub_nodes():
     dst = np.concatenate([np.zeros(700, int), rng.integers(2, 30, 700), rng.integers(2, 30, 300)])
     keep = src != dst
     _run_and_compare(SPEC, "f64", N, src[keep], dst[keep], seed=1)
+    _run_and_compare(("2x0e+3x1o", 2, "3x0e+2x1o+2x2e", 3, "uvw"), "f64", N, src[keep], dst[keep], seed=1)
 
 
 @pytest.mark.parametrize("spec,dtype", [
@@ -78,6 +81,9 @@ def test_isolated_and_hub_nodes():
     (("80x0e+80x1o", 1, "80x0e+80x1o+80x1e", 16, "uvu"), "f64"),       # 3 channel tiles
     (("96x0e+96x1o+96x2e", 2, "96x0e+96x1o+96x2e", 16, "uvu"), "f32"), # K 16, CPL 2, 2 tiles
     (("4x0e+4x1o+4x2e+4x3o+4x4e", 4, "4x0e+4x1o+4x2e+4x3o+4x4e", 3, "uvu"), "f64"),  # l = 4
+    (("2x0e+3x1o", 2, "3x0e+2x1o+2x2e", 3, "uvw"), "f64"),               # uvw, unequal muls
+    (("40x0e+8x1o+5x2e", 2, "7x0e+40x1o+3x1e+9x2e", 16, "uvw"), "f32"),  # uvw, mul > 32
+    (("6x0e+6x1o+6x2e+6x3o+6x4e", 4, "6x0e+6x1o+6x2e+6x3o+6x4e+6x4o", 11, "uvw"), "f64"),
 ])
 def test_shapes(spec, dtype):
     rng = np.random.default_rng(8)

@@ -17,7 +17,7 @@ from oracle import csr as ocsr
 pytestmark = pytest.mark.gpu
 
 # (config, nodes or None for the full workload): small enough for the oracle
-CASES = [(1, None), (3, None), (2, 384), (4, 1500)]
+CASES = [(1, None), (3, None), (2, 384), (4, 1500), (5, 400)]
 
 
 def _check_csr(run):
@@ -57,7 +57,7 @@ def tpc_error():
     return tpc.tp_get_device_error()
 
 
-@pytest.mark.parametrize("cid", [1, 4])
+@pytest.mark.parametrize("cid", [1, 4, 5])
 def test_bitwise_reproducible(cid):
     wl = workload(cid, n_nodes=None if cid == 1 else 1200)
     run = GpuRun(plan_for(cid), wl)
@@ -70,7 +70,7 @@ def test_bitwise_reproducible(cid):
         assert torch.equal(u, v)
 
 
-@pytest.mark.parametrize("cid", [2, 4])
+@pytest.mark.parametrize("cid", [2, 4, 5])
 def test_full_size_sampled(cid):
     """Full-size workload in the benchmark's launch configuration: forward rows of
     sampled receivers, grad_phi/grad_Y of their edges and grad_x of sampled
