@@ -174,6 +174,16 @@ def time_steps(step, steps: int, warmup: int, flush, sampler=None, dist=None):
     return [a.elapsed_time(b) for a, b in evs], clocks
 
 
+def roofline_fb(d, ms: float) -> dict:
+    f0, b0 = d["plan"].work_model(d["N"], d["E"], 0)
+    f1, b1 = d["plan"].work_model(d["N"], d["E"], 1)
+    r = roofline(d, 0, ms)
+    ach = (f0 + f1) / (ms * 1e-3) / 1e12
+    r.update({"achieved": round(ach, 3), "frac": round(ach / r["peak"], 4), "algorithmic_flops": f0 + f1,
+              "compulsory_bytes": b0 + b1})
+    return r
+
+
 def roofline(d, pass_: int, ms: float) -> dict:
     flops, nbytes = d["plan"].work_model(d["N"], d["E"], pass_)
     dt = d["cfg"].dtype
@@ -255,7 +265,14 @@ def run_ours(args, rank, world, dist):
     d = setup(args.config, dev)
     c = d["cfg"]
     sampler = ClockSampler() if rank == 0 else None
-    times, clocks = time_steps(lambda: fwd(d), args.steps, args.warmup, flush, sampler, dist)
+    both = args.pass_ == "fwdbwd"
+
+    def step():
+        fwd(d)
+        if both:
+            bwd(d)
+
+    times, clocks = time_steps(step, args.steps, args.warmup, flush, sampler, dist)
     t_total = sum(times)
     if dist is not None:
         tt = torch.tensor([t_total], dtype=torch.float64, device=dev)
@@ -269,12 +286,14 @@ def run_ours(args, rank, world, dist):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": c.dtype,
            "data": "synthetic",
-           "config": {"workload": c.name, "pass": "forward", "n_nodes": d["N"], "n_edges": d["E"],
+           "config": {"workload": c.name, "pass": "forward+backward" if both else "forward",
+                      "n_nodes": d["N"], "n_edges": d["E"],
                       "irreps_in": c.irreps_in, "irreps_out": c.irreps_out, "sh_lmax": c.sh_lmax,
                       "n_radial": c.K, "mode": c.mode, "parallelism": f"replicas x{world}",
                       "l2": "flushed between steps (256 MiB write outside the timed events)"},
-           "gpu_launches": args.steps,
-           "roofline": roofline(d, 0, ms), "clocks": clocks}
+           "gpu_launches": args.steps * (d["plan"].launch_count(d["N"], 0)
+                                         + (d["plan"].launch_count(d["N"], 1) if both else 0)),
+           "roofline": roofline(d, 0, ms) if not both else roofline_fb(d, ms), "clocks": clocks}
     # end to end through the public API: pinned host inputs -> device -> forward -> host result
     res["e2e"] = e2e(d, args, dev)
     if rank == 0 and not args.no_extra:
@@ -358,6 +377,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "fwdbwd"])
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -91,6 +91,11 @@ class Plan:
               "tp_conv_workspace_size")
         return out.value
 
+    def launch_count(self, n_nodes: int, pass_: int) -> int:
+        out = ctypes.c_int()
+        check(lib().tp_conv_launch_count(self._h, n_nodes, pass_, ctypes.byref(out)), "tp_conv_launch_count")
+        return out.value
+
     def work_model(self, n_nodes: int, n_edges: int, pass_: int) -> Tuple[float, float]:
         f, b = ctypes.c_double(), ctypes.c_double()
         check(lib().tp_conv_work_model(self._h, n_nodes, n_edges, pass_, ctypes.byref(f), ctypes.byref(b)),

@@ -40,6 +40,7 @@ SIGNATURES = {
                                 POINTER(c_double), c_int]),
     "tp_conv_work_model": (c_int, [c_void_p, c_int64, c_int64, c_int, POINTER(c_double), POINTER(c_double)]),
     "tp_conv_workspace_size": (c_int, [c_void_p, c_int64, c_int, POINTER(c_size_t)]),
+    "tp_conv_launch_count": (c_int, [c_void_p, c_int64, c_int, POINTER(c_int)]),
     "tp_csr_workspace_size": (c_int, [c_int64, POINTER(c_size_t)]),
     "tp_csr_build": (c_int, [c_int64, c_int64, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                              c_void_p, c_size_t, c_void_p]),

@@ -423,6 +423,30 @@ int tp_conv_workspace_size(tp_plan_t plan, int64_t n_nodes, int pass, size_t* by
   return TP_OK;
 }
 
+int tp_conv_launch_count(tp_plan_t plan, int64_t n_nodes, int pass, int* kernels) {
+  if (!plan || !kernels) return fail(TP_EINVAL, "NULL argument");
+  if (pass != 0 && pass != 1) return fail(TP_EINVAL, "pass must be 0 or 1");
+  if (n_nodes < 0) return fail(TP_EINVAL, "negative node count");
+  const Plan& P = plan->p;
+  if (n_nodes == 0) {
+    *kernels = 0;
+    return TP_OK;
+  }
+  if (P.mode == TP_UVU) {
+    *kernels = pass == 0 ? 1 : 3;   // forward; edge pass, source pass, grad_A reduction
+    return TP_OK;
+  }
+  const long long nr = uvw_chunk_rows(P, n_nodes, 0), ns = uvw_chunk_rows(P, n_nodes, 1);
+  const long long cr = (n_nodes + nr - 1) / nr, cs = (n_nodes + ns - 1) / ns;
+  const long long gout = ((long long)P.uvw_out.size() + kMaxGemmBatch - 1) / kMaxGemmBatch;
+  const long long gin = ((long long)P.uvw_in.size() + kMaxGemmBatch - 1) / kMaxGemmBatch;
+  if (pass == 0)
+    *kernels = (int)(1 + cr * (1 + gout));                       // pack A; per chunk: state, mixing
+  else
+    *kernels = (int)(1 + cr * (1 + 2 * gout + 1) + cs * (1 + gin) + 1);
+  return TP_OK;
+}
+
 int tp_csr_workspace_size(int64_t n_nodes, size_t* bytes) {
   if (!bytes || n_nodes < 0) return fail(TP_EINVAL, "bad argument");
   *bytes = csr_workspace_bytes(n_nodes);

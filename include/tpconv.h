@@ -136,6 +136,12 @@ int tp_conv_work_model(tp_plan_t plan, int64_t n_nodes, int64_t n_edges, int pas
  * §3.4, Table 2: tensor-product workspace is bounded, not edge-sized). */
 int tp_conv_workspace_size(tp_plan_t plan, int64_t n_nodes, int pass, size_t* bytes);
 
+/* Number of kernels that one tp_conv_forward (pass 0) or tp_conv_backward
+ * (pass 1) call enqueues for n_nodes receivers (memsets not counted). The
+ * fully connected path works on receiver chunks of a fixed state budget, so
+ * its count grows with n_nodes. Host only. */
+int tp_conv_launch_count(tp_plan_t plan, int64_t n_nodes, int pass, int* kernels);
+
 /* Workspace bytes of tp_csr_build / tp_csr_transpose for n_nodes rows. */
 int tp_csr_workspace_size(int64_t n_nodes, size_t* bytes);
 
