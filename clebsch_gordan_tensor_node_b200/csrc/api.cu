@@ -6,6 +6,7 @@
 
 #include "cg_host.h"
 #include "kernels.h"
+#include "launch.h"
 #include "plan.h"
 #include "tpconv.h"
 
@@ -105,10 +106,6 @@ cudaError_t fwd_dispatch(const Plan& P, const UvuFwdParams<T>& p, cudaStream_t s
 }
 
 template <typename T, int KP, int CPL>
-struct EdgeL {
-  static cudaError_t run(const UvuEdgeParams<T>& p, cudaStream_t s) { return launch_uvu_edge<T, KP, CPL>(p, s); }
-};
-template <typename T, int KP, int CPL>
 struct SrcL {
   static cudaError_t run(const UvuSrcParams<T>& p, cudaStream_t s) { return launch_uvu_src<T, KP, CPL>(p, s); }
 };
@@ -142,7 +139,7 @@ int backward_uvu(const Plan& P, const void* x, const void* Y, const void* phi, c
   ep.n_w = (int)P.n_w; ep.n_paths = (int)P.paths_canon.size();
   std::memset(ep.paths, 0, sizeof(ep.paths));
   std::memcpy(ep.paths, P.paths_canon.data(), P.paths_canon.size() * sizeof(PathD));
-  cudaError_t e = dispatch_kc<T, EdgeL>(P, ep, s);
+  cudaError_t e = launch_uvu_edge_for<T>(P, ep, s);
   if (e != cudaSuccess) return cuda_fail(e, "uvu edge pass launch");
 
   UvuSrcParams<T> sp;

@@ -10,8 +10,9 @@ namespace tpc {
 template <typename T, int KP, int CPL, int L1M, int L2M, int L3M>
 cudaError_t launch_uvu_fwd(const UvuFwdParams<T>& p, cudaStream_t s);
 
-template <typename T, int KP, int CPL>
-cudaError_t launch_uvu_edge(const UvuEdgeParams<T>& p, cudaStream_t s);
+// V: channels per 16-byte (fp32: 4) or 8/16-byte (fp64: 2) gather; prof: degree profile
+template <typename T, int KP, int V>
+cudaError_t launch_uvu_edge(const UvuEdgeParams<T>& p, int prof, cudaStream_t s);
 
 template <typename T, int KP, int CPL>
 cudaError_t launch_uvu_src(const UvuSrcParams<T>& p, cudaStream_t s);

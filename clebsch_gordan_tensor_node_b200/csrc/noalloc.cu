@@ -18,6 +18,7 @@
 #include <string>
 
 #include "kernels.h"
+#include "launch.h"
 #include "plan.h"
 #include "tpconv.h"
 
@@ -60,17 +61,6 @@ int scratch_address(void** out) {
 }
 
 template <typename T>
-cudaError_t launch_edge(const Plan& P, const UvuEdgeParams<T>& p, cudaStream_t s) {
-  if (P.KP == 8 && P.CPL == 1) return launch_uvu_edge<T, 8, 1>(p, s);
-  if (P.KP == 16 && P.CPL == 1) return launch_uvu_edge<T, 16, 1>(p, s);
-  if constexpr (std::is_same<T, float>::value) {
-    if (P.KP == 8 && P.CPL == 2) return launch_uvu_edge<T, 8, 2>(p, s);
-    if (P.KP == 16 && P.CPL == 2) return launch_uvu_edge<T, 16, 2>(p, s);
-  }
-  return cudaErrorInvalidValue;
-}
-
-template <typename T>
 cudaError_t launch_src(const Plan& P, const UvuSrcParams<T>& p, cudaStream_t s) {
   if (P.KP == 8 && P.CPL == 1) return launch_uvu_src<T, 8, 1>(p, s);
   if (P.KP == 16 && P.CPL == 1) return launch_uvu_src<T, 16, 1>(p, s);
@@ -94,7 +84,7 @@ int run(const Plan& P, const void* x, const void* Y, const void* phi, const void
   ep.n_w = (int)P.n_w; ep.n_paths = (int)P.paths_canon.size();
   std::memset(ep.paths, 0, sizeof(ep.paths));
   std::memcpy(ep.paths, P.paths_canon.data(), P.paths_canon.size() * sizeof(PathD));
-  cudaError_t e = launch_edge<T>(P, ep, s);
+  cudaError_t e = launch_uvu_edge_for<T>(P, ep, s);
   if (e != cudaSuccess) return set_error_message(TP_ECUDA, std::string("edge pass: ") + cudaGetErrorString(e));
 
   UvuSrcParams<T> sp;

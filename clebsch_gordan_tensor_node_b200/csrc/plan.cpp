@@ -183,6 +183,14 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
     }
   // backward kernels: 1 or 2 channels per lane (fp32), 1 (fp64)
   P.CPL = (dtype == TP_F32 && all_even) ? 2 : 1;
+  // edge pass: 16-byte gathers when every multiplicity allows them
+  {
+    const int vw = dtype == TP_F32 ? 4 : 2;
+    bool ok = true;
+    for (const auto* v : {&P.bin, &P.bout})
+      for (auto& b : *v) ok &= (b.mul % vw == 0);
+    P.edge_V = ok ? vw : 1;
+  }
   // forward: vector width by dtype and block width (every access CPL-aligned);
   // 4 channels per lane measured slower than 2 on the 128-channel workload
   if (dtype == TP_F32)

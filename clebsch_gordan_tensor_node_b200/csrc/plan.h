@@ -25,6 +25,7 @@ struct Plan {
   int dtype = 0;    // 0 f32, 1 f64
   int K = 0, KP = 0, CPL = 1, sh_lmax = 0, lmax = 0;
   int fwd_CPL = 1;          // channels per lane of the forward kernel
+  int edge_V = 1;           // channels per gather in the uvu backward edge pass
   int prof = 3;             // forward degree profile: 0 (2,2,2) 1 (1,3,3) 2 (3,3,3) 3 (4,4,4)
   int cy_stride = 0, fwd_chunk = 32, fwd_warp_smem = 0;
   std::vector<Block> bin, bout;

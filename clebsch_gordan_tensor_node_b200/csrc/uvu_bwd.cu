@@ -27,54 +27,81 @@ namespace {
 constexpr int kDY = (kLmax + 1) * (kLmax + 1);
 
 // ---------------------------------------------------------------- edge pass
+//
+// One lane owns one edge: a warp takes 32 consecutive CSR edges (of any
+// receivers), so phi_bar_e and Y_bar_e accumulate in the owning lane's
+// registers over every path and channel and need no cross-lane reduction. Per
+// path the lane contracts its Y block with the CG pairs once (cY); the channel
+// loop then reads A as a warp-uniform 16-byte broadcast and x_j, m_bar_i as
+// per-lane 16-byte gathers, V channels at a time.
 
-template <typename T, int KP, int CPL, int L1, int L2, int L3>
-__device__ __forceinline__ void edge_path(const UvuEdgeParams<T>& p, const PathD& pd, int lane,
-                                          const T* xrow, const T* grow, const T (&ph)[KP],
-                                          const T (&yall)[kDY], T (&gphi)[KP], T (&gY)[kDY]) {
+template <int L1M, int L2M, int L3M>
+struct Prof {
+  static constexpr int l1 = L1M, l2 = L2M, l3 = L3M;
+};
+
+template <int V, typename T>
+__device__ __forceinline__ void ldv(T (&v)[V], const T* p) {
+  if constexpr (V == 4 && sizeof(T) == 4) {
+    const float4 t = __ldg(reinterpret_cast<const float4*>(p));
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+  } else if constexpr (V == 2 && sizeof(T) == 8) {
+    const double2 t = __ldg(reinterpret_cast<const double2*>(p));
+    v[0] = t.x; v[1] = t.y;
+  } else if constexpr (V == 2 && sizeof(T) == 4) {
+    const float2 t = __ldg(reinterpret_cast<const float2*>(p));
+    v[0] = t.x; v[1] = t.y;
+  } else {
+#pragma unroll
+    for (int c = 0; c < V; ++c) v[c] = __ldg(p + c);
+  }
+}
+
+template <typename T, int KP, int V, int DY, int L1, int L2, int L3>
+__device__ __forceinline__ void edge_path(const UvuEdgeParams<T>& p, const PathD& pd, int e, int j, int i,
+                                          const T (&ph)[KP], T (&gphi)[KP], T (&gY)[DY]) {
   using CGp = cgt::CG<L1, L2, L3>;
-  constexpr int D1 = 2 * L1 + 1, D3 = 2 * L3 + 1, Y0 = L2 * L2;
+  constexpr int D1 = 2 * L1 + 1, D2 = 2 * L2 + 1, D3 = 2 * L3 + 1, NP = CGp::npair, Y0 = L2 * L2;
+  T y[D2];
+#pragma unroll
+  for (int m = 0; m < D2; ++m) y[m] = ldg(p.Y + (size_t)e * p.dim_y + Y0 + m);
+  T cy[NP];
+  static_for<NP>([&](auto P) { cy[decltype(P)::value] = pair_coef<T, CGp, decltype(P)::value>(y); });
   const int mul = pd.mul_in;
-  for (int ch0 = 0; ch0 < mul; ch0 += 32 * CPL) {
-    const bool active = ch0 + lane * CPL < mul;
-    const int chl = ch0 + (active ? lane * CPL : 0);
-    T a[KP][CPL], xv[D1][CPL], gv[D3][CPL];
+  const T* xr = p.x + (size_t)j * p.c_in + pd.x_off;
+  const T* gr = p.gout + (size_t)i * p.c_out + pd.out_off;
+  const T* ar = p.A + pd.w_off;
+  for (int u0 = 0; u0 < mul; u0 += V) {
+    T a[KP][V], xv[D1][V], gv[D3][V];
 #pragma unroll
     for (int q = 0; q < KP; ++q) {
       if (q < p.K) {
-        load_ch<CPL>(a[q], p.A + (size_t)q * p.n_w + pd.w_off + chl);
+        ldv<V>(a[q], ar + (size_t)q * p.n_w + u0);
       } else {
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) a[q][c] = T(0);
+        for (int c = 0; c < V; ++c) a[q][c] = T(0);
       }
     }
 #pragma unroll
-    for (int m = 0; m < D1; ++m) load_ch<CPL>(xv[m], xrow + pd.x_off + m * mul + chl);
+    for (int m = 0; m < D1; ++m) ldv<V>(xv[m], xr + m * mul + u0);
 #pragma unroll
-    for (int m = 0; m < D3; ++m) load_ch<CPL>(gv[m], grow + pd.out_off + m * pd.mul_out + chl);
-    if (!active) {
+    for (int m = 0; m < D3; ++m) ldv<V>(gv[m], gr + m * mul + u0);
+    T w[V], h[V];
 #pragma unroll
-      for (int m = 0; m < D1; ++m)
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) xv[m][c] = T(0);
-    }
-    T w[CPL], h[CPL];
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) {
+    for (int c = 0; c < V; ++c) {
       w[c] = ph[0] * a[0][c];
 #pragma unroll
       for (int q = 1; q < KP; ++q) w[c] = fma(ph[q], a[q][c], w[c]);
       h[c] = T(0);
     }
-    static_for<CGp::npair>([&](auto P) {
+    static_for<NP>([&](auto P) {
       constexpr int Pi = decltype(P)::value;
       constexpr Pair pr = CGp::pair[Pi];
-      const T cy = pair_coef<T, CGp, Pi>(yall + Y0);
       T z = T(0);
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) {
+      for (int c = 0; c < V; ++c) {
         const T xg = xv[pr.m1][c] * gv[pr.m3][c];
-        h[c] = fma(cy, xg, h[c]);
+        h[c] = fma(cy[Pi], xg, h[c]);
         z = fma(w[c], xg, z);
       }
       // Y_bar[m2] += c * sum_u w x[m1] m_bar[m3]
@@ -86,70 +113,70 @@ __device__ __forceinline__ void edge_path(const UvuEdgeParams<T>& p, const PathD
 #pragma unroll
     for (int q = 0; q < KP; ++q)
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) gphi[q] = fma(a[q][c], h[c], gphi[q]);
+      for (int c = 0; c < V; ++c) gphi[q] = fma(a[q][c], h[c], gphi[q]);
   }
 }
 
-template <typename T>
-__device__ __forceinline__ T warp_sum(T v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
-template <typename T, int KP, int CPL>
+template <typename T, int KP, int V, class PR>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 uvu_edge_kernel(const __grid_constant__ UvuEdgeParams<T> p) {
+  constexpr int DY = (PR::l2 + 1) * (PR::l2 + 1);
   const int lane = threadIdx.x & 31;
-  const int i = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
-  if (i >= p.N) return;
-  int e0 = ldg(p.rowptr + i), e1 = ldg(p.rowptr + i + 1);
-  if (e0 < 0 || e1 < e0 || e1 > p.E) {
-    raise_error(p.err, kErrCsr);
-    return;
+  const long long e0 = ((long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5)) * 32;
+  if (e0 >= p.E) return;
+  const int e = (int)(e0 + lane);
+  const bool live = e < p.E;
+  // receiver of CSR position e: the last i with rowptr[i] <= e
+  int i = 0;
+  int j = 0;
+  bool ok = false;
+  if (live) {
+    int lo = 0, hi = p.N;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (ldg(p.rowptr + mid) <= e) lo = mid; else hi = mid;
+    }
+    i = lo;
+    j = ldg(p.senders + e);
+    ok = (unsigned)j < (unsigned)p.N;
+    if (!ok) atomicOr(p.err, kErrIndex);
+    if (!ok) j = 0;
   }
-  const T* grow = p.gout + (size_t)i * p.c_out;
-  for (int e = e0; e < e1; ++e) {
-    const int j = ldg(p.senders + e);
-    T gphi[KP], gY[kDY];
+  T ph[KP], gphi[KP], gY[DY];
 #pragma unroll
-    for (int q = 0; q < KP; ++q) gphi[q] = T(0);
+  for (int q = 0; q < KP; ++q) {
+    ph[q] = (live && q < p.K) ? ldg(p.phi + (size_t)e * p.K + q) : T(0);
+    gphi[q] = T(0);
+  }
 #pragma unroll
-    for (int m = 0; m < kDY; ++m) gY[m] = T(0);
-    if ((unsigned)j < (unsigned)p.N) {
-      T ph[KP], yall[kDY];
-      load_phi<KP>(ph, p.phi + (size_t)e * p.K, p.K);
-#pragma unroll
-      for (int m = 0; m < kDY; ++m) yall[m] = m < p.dim_y ? ldg(p.Y + (size_t)e * p.dim_y + m) : T(0);
-      const T* xrow = p.x + (size_t)j * p.c_in;
-      for (int pi = 0; pi < p.n_paths; ++pi) {
-        const PathD& pd = p.paths[pi];
-        dispatch_l(pd.l1, [&](auto A1) {
-          constexpr int L1 = decltype(A1)::value;
-          dispatch_l2l3<L1>(pd.l2, pd.l3, [&](auto A2, auto A3) {
-            edge_path<T, KP, CPL, L1, decltype(A2)::value, decltype(A3)::value>(
-                p, pd, lane, xrow, grow, ph, yall, gphi, gY);
+  for (int m = 0; m < DY; ++m) gY[m] = T(0);
+  if (live) {
+    for (int pi = 0; pi < p.n_paths; ++pi) {
+      const PathD& pd = p.paths[pi];
+      dispatch_l<PR::l1>(pd.l1, [&](auto A1) {
+        constexpr int L1 = decltype(A1)::value;
+        static_for<PR::l2 + 1>([&](auto A2) {
+          static_for<PR::l3 + 1>([&](auto A3) {
+            constexpr int L2 = decltype(A2)::value, L3 = decltype(A3)::value;
+            if constexpr (triangle(L1, L2, L3)) {
+              if (pd.l2 == L2 && pd.l3 == L3) edge_path<T, KP, V, DY, L1, L2, L3>(p, pd, e, j, i, ph, gphi, gY);
+            }
           });
         });
-      }
-    } else {
-      raise_error(p.err, kErrIndex);
+      });
     }
-    // one reduction per edge; lane 0 writes
+    if (!ok) {
 #pragma unroll
-    for (int q = 0; q < KP; ++q) {
-      if (q < p.K) {
-        const T v = warp_sum(gphi[q]);
-        if (lane == 0) p.gphi[(size_t)e * p.K + q] = v;
-      }
+      for (int q = 0; q < KP; ++q) gphi[q] = T(0);
+#pragma unroll
+      for (int m = 0; m < DY; ++m) gY[m] = T(0);
     }
 #pragma unroll
-    for (int m = 0; m < kDY; ++m) {
-      if (m < p.dim_y) {
-        const T v = warp_sum(gY[m]);
-        if (lane == 0) p.gY[(size_t)e * p.dim_y + m] = v;
-      }
-    }
+    for (int q = 0; q < KP; ++q)
+      if (q < p.K) p.gphi[(size_t)e * p.K + q] = gphi[q];
+#pragma unroll
+    for (int m = 0; m < DY; ++m)
+      if (m < p.dim_y) p.gY[(size_t)e * p.dim_y + m] = gY[m];
   }
 }
 
@@ -298,11 +325,17 @@ __global__ void reduce_slots_kernel(const T* __restrict__ part, T* __restrict__ 
 
 }  // namespace
 
-template <typename T, int KP, int CPL>
-cudaError_t launch_uvu_edge(const UvuEdgeParams<T>& p, cudaStream_t s) {
-  if (p.N == 0) return cudaSuccess;
-  const int blocks = (p.N + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  uvu_edge_kernel<T, KP, CPL><<<blocks, kWarpsPerBlock * 32, 0, s>>>(p);
+template <typename T, int KP, int V>
+cudaError_t launch_uvu_edge(const UvuEdgeParams<T>& p, int prof, cudaStream_t s) {
+  if (p.N == 0 || p.E == 0) return cudaSuccess;
+  const long long warps = ((long long)p.E + 31) / 32;
+  const unsigned blocks = (unsigned)((warps + kWarpsPerBlock - 1) / kWarpsPerBlock);
+  switch (prof) {
+    case 0: uvu_edge_kernel<T, KP, V, Prof<2, 2, 2>><<<blocks, kWarpsPerBlock * 32, 0, s>>>(p); break;
+    case 1: uvu_edge_kernel<T, KP, V, Prof<1, 3, 3>><<<blocks, kWarpsPerBlock * 32, 0, s>>>(p); break;
+    case 2: uvu_edge_kernel<T, KP, V, Prof<3, 3, 3>><<<blocks, kWarpsPerBlock * 32, 0, s>>>(p); break;
+    default: uvu_edge_kernel<T, KP, V, Prof<4, 4, 4>><<<blocks, kWarpsPerBlock * 32, 0, s>>>(p); break;
+  }
   return cudaGetLastError();
 }
 
@@ -324,28 +357,44 @@ cudaError_t launch_reduce_slots(const T* part, T* out, int n_slots, long long n,
   return cudaGetLastError();
 }
 
-#define TPC_INST(T, KP, CPL)                                                                   \
-  template cudaError_t launch_uvu_edge<T, KP, CPL>(const UvuEdgeParams<T>&, cudaStream_t);     \
+#define TPC_INST_SRC(T, KP, CPL) \
   template cudaError_t launch_uvu_src<T, KP, CPL>(const UvuSrcParams<T>&, cudaStream_t);
+#define TPC_INST_EDGE(T, KP, V) \
+  template cudaError_t launch_uvu_edge<T, KP, V>(const UvuEdgeParams<T>&, int, cudaStream_t);
 #if TPC_WANT(0)
-TPC_INST(float, 8, 1)
+TPC_INST_SRC(float, 8, 1)
+TPC_INST_SRC(float, 8, 2)
 #endif
 #if TPC_WANT(1)
-TPC_INST(float, 8, 2)
+TPC_INST_SRC(float, 16, 1)
+TPC_INST_SRC(float, 16, 2)
 #endif
 #if TPC_WANT(2)
-TPC_INST(float, 16, 1)
+TPC_INST_SRC(double, 8, 1)
+TPC_INST_SRC(double, 16, 1)
 #endif
 #if TPC_WANT(3)
-TPC_INST(float, 16, 2)
+TPC_INST_EDGE(float, 8, 1)
 #endif
 #if TPC_WANT(4)
-TPC_INST(double, 8, 1)
+TPC_INST_EDGE(float, 8, 4)
 #endif
 #if TPC_WANT(5)
-TPC_INST(double, 16, 1)
+TPC_INST_EDGE(float, 16, 1)
+TPC_INST_EDGE(float, 16, 4)
 #endif
-#undef TPC_INST
+#if TPC_WANT(6)
+TPC_INST_EDGE(double, 8, 1)
+#endif
+#if TPC_WANT(7)
+TPC_INST_EDGE(double, 8, 2)
+#endif
+#if TPC_WANT(8)
+TPC_INST_EDGE(double, 16, 1)
+TPC_INST_EDGE(double, 16, 2)
+#endif
+#undef TPC_INST_SRC
+#undef TPC_INST_EDGE
 #if TPC_WANT(0)
 template cudaError_t launch_reduce_slots<float>(const float*, float*, int, long long, cudaStream_t);
 template cudaError_t launch_reduce_slots<double>(const double*, double*, int, long long, cudaStream_t);
