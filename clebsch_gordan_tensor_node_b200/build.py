@@ -26,7 +26,7 @@ CG_LMAX = 6
 # translation units and how many instantiation sets each one is split into
 UNITS = {
     "uvu_fwd.cu": 9,
-    "uvu_bwd.cu": 9,
+    "uvu_bwd.cu": 10,
     "uvw.cu": 4,
     "gemm.cu": 1,
     "csr.cu": 1,

@@ -68,17 +68,6 @@ void copy_tables(P& prm, const std::vector<TileD>& tiles, const std::vector<Path
   prm.n_tiles = (int)tiles.size();
 }
 
-template <typename T, template <typename, int, int> class L, typename Prm>
-cudaError_t dispatch_kc(const Plan& P, const Prm& prm, cudaStream_t s) {
-  if (P.KP == 8 && P.CPL == 1) return L<T, 8, 1>::run(prm, s);
-  if (P.KP == 16 && P.CPL == 1) return L<T, 16, 1>::run(prm, s);
-  if constexpr (std::is_same<T, float>::value) {
-    if (P.KP == 8 && P.CPL == 2) return L<T, 8, 2>::run(prm, s);
-    if (P.KP == 16 && P.CPL == 2) return L<T, 16, 2>::run(prm, s);
-  }
-  return cudaErrorInvalidValue;
-}
-
 template <typename T, int KP, int CPL, bool Full>
 cudaError_t fwd_prof(const Plan& P, const UvuFwdParams<T>& p, cudaStream_t s) {
   switch (P.prof) {
@@ -105,10 +94,6 @@ cudaError_t fwd_dispatch(const Plan& P, const UvuFwdParams<T>& p, cudaStream_t s
   return cudaErrorInvalidValue;
 }
 
-template <typename T, int KP, int CPL>
-struct SrcL {
-  static cudaError_t run(const UvuSrcParams<T>& p, cudaStream_t s) { return launch_uvu_src<T, KP, CPL>(p, s); }
-};
 
 template <typename T>
 int forward_uvu(const Plan& P, const void* x, const void* Y, const void* phi, const void* A,
@@ -150,7 +135,7 @@ int backward_uvu(const Plan& P, const void* x, const void* Y, const void* phi, c
   sp.n_w = (int)P.n_w;
   sp.n_slots = uvu_src_slots(P, N);
   copy_tables(sp, P.in_tiles, P.paths_by_in);
-  e = dispatch_kc<T, SrcL>(P, sp, s);
+  e = launch_uvu_src_for<T>(P, sp, s);
   if (e != cudaSuccess) return cuda_fail(e, "uvu source pass launch");
   e = launch_reduce_slots<T>((const T*)ws, (T*)gA, sp.n_slots, (long long)P.K * P.n_w, s);
   return e == cudaSuccess ? TP_OK : cuda_fail(e, "grad_A reduction launch");

@@ -78,6 +78,9 @@ struct UvuSrcParams {         // backward: source-owned grad_x, grad_A partials
   T* gx; T* apart; int* err;
   int N, E, K, c_in, c_out, dim_y, n_w;
   int n_tiles, n_slots;
+  int cy_stride;              // cY slots per staged edge (max over tiles, padded)
+  int chunk;                  // edges staged per warp at a time (<= 32)
+  int warp_smem;              // bytes of shared memory per warp
   TileD tiles[kMaxTiles];     // one per (input block, channel tile)
   PathD paths[kMaxPaths];     // grouped by input block
 };

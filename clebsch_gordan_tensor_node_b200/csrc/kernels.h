@@ -15,7 +15,7 @@ template <typename T, int KP, int V>
 cudaError_t launch_uvu_edge(const UvuEdgeParams<T>& p, int prof, cudaStream_t s);
 
 template <typename T, int KP, int CPL>
-cudaError_t launch_uvu_src(const UvuSrcParams<T>& p, cudaStream_t s);
+cudaError_t launch_uvu_src(const UvuSrcParams<T>& p, int prof, cudaStream_t s);
 
 template <typename T>
 cudaError_t launch_reduce_slots(const T* part, T* out, int n_slots, long long n, cudaStream_t s);

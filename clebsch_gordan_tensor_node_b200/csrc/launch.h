@@ -21,4 +21,16 @@ cudaError_t launch_uvu_edge_for(const Plan& P, const UvuEdgeParams<T>& p, cudaSt
   return launch_uvu_edge<T, 16, 1>(p, P.prof, s);
 }
 
+// Source pass of the uvu backward: radial width KP, channels per lane, profile.
+template <typename T>
+cudaError_t launch_uvu_src_for(const Plan& P, UvuSrcParams<T>& p, cudaStream_t s) {
+  p.cy_stride = P.src_cy_stride;
+  p.chunk = P.src_chunk;
+  p.warp_smem = P.src_warp_smem;
+  if constexpr (std::is_same<T, float>::value) {
+    if (P.CPL == 2) return P.KP == 8 ? launch_uvu_src<T, 8, 2>(p, P.prof, s) : launch_uvu_src<T, 16, 2>(p, P.prof, s);
+  }
+  return P.KP == 8 ? launch_uvu_src<T, 8, 1>(p, P.prof, s) : launch_uvu_src<T, 16, 1>(p, P.prof, s);
+}
+
 }  // namespace tpc

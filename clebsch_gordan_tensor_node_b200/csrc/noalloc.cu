@@ -61,17 +61,6 @@ int scratch_address(void** out) {
 }
 
 template <typename T>
-cudaError_t launch_src(const Plan& P, const UvuSrcParams<T>& p, cudaStream_t s) {
-  if (P.KP == 8 && P.CPL == 1) return launch_uvu_src<T, 8, 1>(p, s);
-  if (P.KP == 16 && P.CPL == 1) return launch_uvu_src<T, 16, 1>(p, s);
-  if constexpr (std::is_same<T, float>::value) {
-    if (P.KP == 8 && P.CPL == 2) return launch_uvu_src<T, 8, 2>(p, s);
-    if (P.KP == 16 && P.CPL == 2) return launch_uvu_src<T, 16, 2>(p, s);
-  }
-  return cudaErrorInvalidValue;
-}
-
-template <typename T>
 int run(const Plan& P, const void* x, const void* Y, const void* phi, const void* A, const int* rowptr,
         const int* senders, const int* colptr, const int* srcedge, const int* srcrecv, const void* gout,
         int N, int E, void* gx, void* gY, void* gphi, void* gA, void* scratch, int slots, int* err,
@@ -101,7 +90,7 @@ int run(const Plan& P, const void* x, const void* Y, const void* phi, const void
   sp.n_tiles = (int)P.in_tiles.size();
   // launch_uvu_src first clears the slots it uses (the scratch keeps the previous
   // call's contents), then accumulates into them
-  e = launch_src<T>(P, sp, s);
+  e = launch_uvu_src_for<T>(P, sp, s);
   if (e != cudaSuccess) return set_error_message(TP_ECUDA, std::string("source pass: ") + cudaGetErrorString(e));
   e = launch_reduce_slots<T>((const T*)scratch, (T*)gA, slots, (long long)P.K * P.n_w, s);
   if (e != cudaSuccess) return set_error_message(TP_ECUDA, std::string("grad_A reduction: ") + cudaGetErrorString(e));

@@ -248,6 +248,25 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
   P.fwd_chunk = std::max(1, std::min(32, (20 * 1024) / (P.cy_stride * bsz)));
   P.fwd_warp_smem = 32 * 4 + 32 * P.KP * bsz + P.fwd_chunk * P.cy_stride * bsz;
   P.fwd_warp_smem = (P.fwd_warp_smem + 15) / 16 * 16;
+  // the same staging for the source pass of the backward (paths by input block)
+  P.src_cy_stride = vw;
+  for (const TileD& t : P.in_tiles) {
+    int off = 0;
+    for (int k = t.pbeg; k < t.pend; ++k) {
+      PathD& d = P.paths_by_in[k];
+      auto e = real_cg_sparse(d.l1, d.l2, d.l3);
+      std::vector<std::pair<int, int>> pairs;
+      for (auto& q : e) pairs.emplace_back(q.m1, q.m3);
+      std::sort(pairs.begin(), pairs.end());
+      pairs.erase(std::unique(pairs.begin(), pairs.end()), pairs.end());
+      d.cy_off = off;
+      off += ((int)pairs.size() + vw - 1) / vw * vw;
+    }
+    P.src_cy_stride = std::max(P.src_cy_stride, off);
+  }
+  P.src_chunk = std::max(1, std::min(32, (20 * 1024) / (P.src_cy_stride * bsz)));
+  P.src_warp_smem = 32 * 4 + 32 * P.KP * bsz + P.src_chunk * P.src_cy_stride * bsz;
+  P.src_warp_smem = (P.src_warp_smem + 15) / 16 * 16;
   if (mode == TP_UVW) {
     if ((int)P.bout.size() > kMaxBlocks || (int)P.bin.size() > kMaxBlocks) {
       msg = "more than " + std::to_string(kMaxBlocks) + " irrep blocks";

@@ -181,13 +181,50 @@ uvu_edge_kernel(const __grid_constant__ UvuEdgeParams<T> p) {
 }
 
 // ---------------------------------------------------------------- source pass
+//
+// The forward's structure on the source view: a warp owns (source j, input
+// block b, channel tile); per chunk of up to 32 outgoing edges, lanes first
+// stage each edge's receiver, radial row and the cY values of every path of b
+// in shared memory; then every path sweeps the chunk with A in registers and
+// the next receiver's m_bar gather in flight. x_bar_j accumulates in registers
+// in one fixed order; the same sweep forms h = <x_j, t'> and adds phi h to the
+// warp's slot of the A_bar partial buffer after each path.
+
+template <typename T>
+struct SrcSmem {
+  int* i;
+  T* phi;
+  T* cy;
+};
+
+template <typename T, int L1, int L2, int L3>
+__device__ __forceinline__ void src_stage_cy(const T* yrow, T* dst) {
+  using CGp = cgt::CG<L1, L2, L3>;
+  T y[2 * L2 + 1];
+#pragma unroll
+  for (int m = 0; m < 2 * L2 + 1; ++m) y[m] = ldg(yrow + L2 * L2 + m);
+  static_for<CGp::npair>([&](auto P) { dst[decltype(P)::value] = pair_coef<T, CGp, decltype(P)::value>(y); });
+}
+
+template <typename T>
+__device__ __forceinline__ void lds16(T* v, const T* src) {
+  if constexpr (sizeof(T) == 4) {
+    const float4 t = *reinterpret_cast<const float4*>(src);
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+  } else {
+    const double2 t = *reinterpret_cast<const double2*>(src);
+    v[0] = t.x; v[1] = t.y;
+  }
+}
 
 template <typename T, int KP, int CPL, int L1, int L2, int L3>
-__device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& pd, int slot,
-                                         int chl, bool active, int k0, int k1,
-                                         const T (&xs)[2 * L1 + 1][CPL], T (&gx)[2 * L1 + 1][CPL]) {
+__device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& pd, const SrcSmem<T>& s, int n,
+                                         int slot, int chl, bool active, const T (&xs)[2 * L1 + 1][CPL],
+                                         T (&gx)[2 * L1 + 1][CPL]) {
   using CGp = cgt::CG<L1, L2, L3>;
-  constexpr int D1 = 2 * L1 + 1, D2 = 2 * L2 + 1, D3 = 2 * L3 + 1;
+  constexpr int D1 = 2 * L1 + 1, D3 = 2 * L3 + 1, NP = CGp::npair;
+  constexpr int VW = sizeof(T) == 4 ? 4 : 2;
+  constexpr bool kPrefetch = D3 * CPL * sizeof(T) <= 48;
   T a[KP][CPL], ab[KP][CPL];
 #pragma unroll
   for (int q = 0; q < KP; ++q) {
@@ -200,21 +237,31 @@ __device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& 
       for (int c = 0; c < CPL; ++c) a[q][c] = T(0);
     }
   }
+  const T* gb = p.gout + pd.out_off + chl;
   const int mo = pd.mul_out;
-  for (int k = k0; k < k1; ++k) {
-    const int e = ldg(p.srcedge + k);
-    const int i = ldg(p.srcrecv + k);
-    if ((unsigned)e >= (unsigned)p.E || (unsigned)i >= (unsigned)p.N) {
-      raise_error(p.err, kErrIndex);
-      continue;
-    }
-    T ph[KP], y[D2], gv[D3][CPL];
-    load_phi<KP>(ph, p.phi + (size_t)e * p.K, p.K);
-#pragma unroll
-    for (int m = 0; m < D2; ++m) y[m] = ldg(p.Y + (size_t)e * p.dim_y + L2 * L2 + m);
-    const T* gr = p.gout + (size_t)i * p.c_out + pd.out_off + chl;
+  T gv[D3][CPL];
+  if (kPrefetch && n > 0) {
+    const T* gr = gb + (size_t)s.i[0] * p.c_out;
 #pragma unroll
     for (int m = 0; m < D3; ++m) load_ch<CPL>(gv[m], gr + m * mo);
+  }
+  for (int k = 0; k < n; ++k) {
+    T gn[kPrefetch ? D3 : 1][CPL];
+    if constexpr (kPrefetch) {
+      if (k + 1 < n) {
+        const T* gr = gb + (size_t)s.i[k + 1] * p.c_out;
+#pragma unroll
+        for (int m = 0; m < D3; ++m) load_ch<CPL>(gn[m], gr + m * mo);
+      }
+    } else {
+      const T* gr = gb + (size_t)s.i[k] * p.c_out;
+#pragma unroll
+      for (int m = 0; m < D3; ++m) load_ch<CPL>(gv[m], gr + m * mo);
+    }
+    T ph[KP];
+#pragma unroll
+    for (int q = 0; q < KP; q += VW) lds16(ph + q, s.phi + k * KP + q);
+    const T* cyr = s.cy + k * p.cy_stride + pd.cy_off;
     T w[CPL];
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
@@ -224,16 +271,17 @@ __device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& 
     }
     // t'[m1] = sum_{m3} cY[m1][m3] m_bar[m3]   (D_x T^* applied to m_bar)
     T tp[D1][CPL];
-    static_for<CGp::npair>([&](auto P) {
+    T cyv[VW];
+    static_for<NP>([&](auto P) {
       constexpr int Pi = decltype(P)::value;
       constexpr Pair pr = CGp::pair[Pi];
-      const T cy = pair_coef<T, CGp, Pi>(y);
+      if constexpr (Pi % VW == 0) lds16(cyv, cyr + Pi);
 #pragma unroll
       for (int c = 0; c < CPL; ++c) {
         if constexpr (first_m1<CGp>(Pi))
-          tp[pr.m1][c] = cy * gv[pr.m3][c];
+          tp[pr.m1][c] = cyv[Pi % VW] * gv[pr.m3][c];
         else
-          tp[pr.m1][c] = fma(cy, gv[pr.m3][c], tp[pr.m1][c]);
+          tp[pr.m1][c] = fma(cyv[Pi % VW], gv[pr.m3][c], tp[pr.m1][c]);
       }
     });
     T h[CPL];
@@ -253,8 +301,16 @@ __device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& 
     for (int q = 0; q < KP; ++q)
 #pragma unroll
       for (int c = 0; c < CPL; ++c) ab[q][c] = fma(ph[q], h[c], ab[q][c]);
+    if constexpr (kPrefetch) {
+      if (k + 1 < n) {
+#pragma unroll
+        for (int m = 0; m < D3; ++m)
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) gv[m][c] = gn[m][c];
+      }
+    }
   }
-  if (active && k1 > k0) {
+  if (active && n > 0) {
 #pragma unroll
     for (int q = 0; q < KP; ++q) {
       if (q < p.K) {
@@ -268,8 +324,9 @@ __device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& 
   }
 }
 
-template <typename T, int KP, int CPL, int L1>
-__device__ __forceinline__ void src_tile(const UvuSrcParams<T>& p, const TileD& tl, int slot, int lane) {
+template <typename T, int KP, int CPL, class PR, int L1>
+__device__ __forceinline__ void src_tile(const UvuSrcParams<T>& p, const TileD& tl, int slot, int lane,
+                                         const SrcSmem<T>& s) {
   constexpr int D1 = 2 * L1 + 1;
   const bool active = lane * CPL < tl.nch;
   const int chl = tl.ch0 + (active ? lane * CPL : 0);
@@ -287,12 +344,42 @@ __device__ __forceinline__ void src_tile(const UvuSrcParams<T>& p, const TileD& 
 #pragma unroll
       for (int c = 0; c < CPL; ++c) gx[m][c] = T(0);
     }
-    for (int pi = tl.pbeg; pi < tl.pend; ++pi) {
-      const PathD& pd = p.paths[pi];
-      dispatch_l2l3<L1>(pd.l2, pd.l3, [&](auto A2, auto A3) {
-        src_path<T, KP, CPL, L1, decltype(A2)::value, decltype(A3)::value>(p, pd, slot, chl, active,
-                                                                           k0, k1, xs, gx);
-      });
+    for (int c0 = k0; c0 < k1; c0 += p.chunk) {
+      const int n = min(p.chunk, k1 - c0);
+      if (lane < n) {
+        const int k = c0 + lane;
+        int e = ldg(p.srcedge + k), i = ldg(p.srcrecv + k);
+        const bool ok = (unsigned)e < (unsigned)p.E && (unsigned)i < (unsigned)p.N;
+        if (!ok) {
+          atomicOr(p.err, kErrIndex);
+          e = 0;
+          i = 0;
+        }
+        s.i[lane] = i;
+        T ph[KP];
+        load_phi<KP>(ph, p.phi + (size_t)e * p.K, p.K);
+#pragma unroll
+        for (int q = 0; q < KP; ++q) s.phi[lane * KP + q] = ok ? ph[q] : T(0);
+        const T* yrow = p.Y + (size_t)e * p.dim_y;
+        T* cyrow = s.cy + lane * p.cy_stride;
+        for (int pi = tl.pbeg; pi < tl.pend; ++pi) {
+          const PathD& pd = p.paths[pi];
+          dispatch_l2l3<L1, PR::l2>(pd.l2, pd.l3, [&](auto A2, auto A3) {
+            if constexpr (decltype(A3)::value <= PR::l3)
+              src_stage_cy<T, L1, decltype(A2)::value, decltype(A3)::value>(yrow, cyrow + pd.cy_off);
+          });
+        }
+      }
+      __syncwarp();
+      for (int pi = tl.pbeg; pi < tl.pend; ++pi) {
+        const PathD& pd = p.paths[pi];
+        dispatch_l2l3<L1, PR::l2>(pd.l2, pd.l3, [&](auto A2, auto A3) {
+          if constexpr (decltype(A3)::value <= PR::l3)
+            src_path<T, KP, CPL, L1, decltype(A2)::value, decltype(A3)::value>(p, pd, s, n, slot, chl, active, xs,
+                                                                               gx);
+        });
+      }
+      __syncwarp();
     }
     if (active) {
       T* o = p.gx + (size_t)j * p.c_in + tl.off + chl;
@@ -302,15 +389,21 @@ __device__ __forceinline__ void src_tile(const UvuSrcParams<T>& p, const TileD& 
   }
 }
 
-template <typename T, int KP, int CPL>
+template <typename T, int KP, int CPL, class PR>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 uvu_src_kernel(const __grid_constant__ UvuSrcParams<T> p) {
-  const int lane = threadIdx.x & 31;
-  const int wid = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int wid = blockIdx.x * kWarpsPerBlock + warp;
   if (wid >= p.n_slots * p.n_tiles) return;
   const int slot = wid / p.n_tiles;
   const TileD& tl = p.tiles[wid % p.n_tiles];
-  dispatch_l(tl.l, [&](auto L) { src_tile<T, KP, CPL, decltype(L)::value>(p, tl, slot, lane); });
+  unsigned char* base = smem_raw + (size_t)warp * p.warp_smem;
+  SrcSmem<T> s;
+  s.i = reinterpret_cast<int*>(base);
+  s.phi = reinterpret_cast<T*>(base + 32 * sizeof(int));
+  s.cy = s.phi + 32 * KP;
+  dispatch_l<PR::l1>(tl.l, [&](auto L) { src_tile<T, KP, CPL, PR, decltype(L)::value>(p, tl, slot, lane, s); });
 }
 
 template <typename T>
@@ -339,15 +432,31 @@ cudaError_t launch_uvu_edge(const UvuEdgeParams<T>& p, int prof, cudaStream_t s)
   return cudaGetLastError();
 }
 
+template <typename T, int KP, int CPL, class PR>
+cudaError_t launch_src_prof(const UvuSrcParams<T>& p, unsigned blocks, cudaStream_t s) {
+  const size_t smem = (size_t)p.warp_smem * kWarpsPerBlock;
+  auto kern = uvu_src_kernel<T, KP, CPL, PR>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<blocks, kWarpsPerBlock * 32, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
 template <typename T, int KP, int CPL>
-cudaError_t launch_uvu_src(const UvuSrcParams<T>& p, cudaStream_t s) {
+cudaError_t launch_uvu_src(const UvuSrcParams<T>& p, int prof, cudaStream_t s) {
   cudaError_t err = cudaMemsetAsync(p.apart, 0, sizeof(T) * (size_t)p.n_slots * p.K * p.n_w, s);
   if (err != cudaSuccess) return err;
   const long long warps = (long long)p.n_slots * p.n_tiles;
   if (warps == 0 || p.N == 0) return cudaSuccess;
-  const long long blocks = (warps + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  uvu_src_kernel<T, KP, CPL><<<(unsigned)blocks, kWarpsPerBlock * 32, 0, s>>>(p);
-  return cudaGetLastError();
+  const unsigned blocks = (unsigned)((warps + kWarpsPerBlock - 1) / kWarpsPerBlock);
+  switch (prof) {
+    case 0: return launch_src_prof<T, KP, CPL, Prof<2, 2, 2>>(p, blocks, s);
+    case 1: return launch_src_prof<T, KP, CPL, Prof<1, 3, 3>>(p, blocks, s);
+    case 2: return launch_src_prof<T, KP, CPL, Prof<3, 3, 3>>(p, blocks, s);
+    default: return launch_src_prof<T, KP, CPL, Prof<4, 4, 4>>(p, blocks, s);
+  }
 }
 
 template <typename T>
@@ -358,18 +467,20 @@ cudaError_t launch_reduce_slots(const T* part, T* out, int n_slots, long long n,
 }
 
 #define TPC_INST_SRC(T, KP, CPL) \
-  template cudaError_t launch_uvu_src<T, KP, CPL>(const UvuSrcParams<T>&, cudaStream_t);
+  template cudaError_t launch_uvu_src<T, KP, CPL>(const UvuSrcParams<T>&, int, cudaStream_t);
 #define TPC_INST_EDGE(T, KP, V) \
   template cudaError_t launch_uvu_edge<T, KP, V>(const UvuEdgeParams<T>&, int, cudaStream_t);
 #if TPC_WANT(0)
 TPC_INST_SRC(float, 8, 1)
-TPC_INST_SRC(float, 8, 2)
 #endif
 #if TPC_WANT(1)
+TPC_INST_SRC(float, 8, 2)
+#endif
+#if TPC_WANT(2)
 TPC_INST_SRC(float, 16, 1)
 TPC_INST_SRC(float, 16, 2)
 #endif
-#if TPC_WANT(2)
+#if TPC_WANT(9)
 TPC_INST_SRC(double, 8, 1)
 TPC_INST_SRC(double, 16, 1)
 #endif
