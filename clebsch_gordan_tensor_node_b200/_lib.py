@@ -14,7 +14,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtpconv.s
 TP_UVU, TP_UVW = 0, 1
 TP_F32, TP_F64 = 0, 1
 STATUS = {0: "TP_OK", -1: "TP_EINVAL", -2: "TP_EUNSUPPORTED", -3: "TP_ECUDA",
-          -4: "TP_EWORKSPACE", -5: "TP_EDEVICE_INDEX", -6: "TP_EDEVICE_CSR"}
+          -4: "TP_EWORKSPACE", -5: "TP_EDEVICE_INDEX", -6: "TP_EDEVICE_CSR", -7: "TP_EDEVICE_TIMEOUT"}
 
 
 class PlanInfo(ctypes.Structure):

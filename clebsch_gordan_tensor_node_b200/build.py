@@ -27,8 +27,9 @@ CG_LMAX = 6
 UNITS = {
     "uvu_fwd.cu": 9,
     "uvu_bwd.cu": 10,
-    "uvw.cu": 4,
+    "uvw.cu": 10,
     "gemm.cu": 1,
+    "tc_gemm.cu": 1,
     "csr.cu": 1,
     "api.cu": 1,
     "noalloc.cu": 1,

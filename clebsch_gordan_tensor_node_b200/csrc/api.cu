@@ -143,9 +143,18 @@ int backward_uvu(const Plan& P, const void* x, const void* Y, const void* phi, c
 
 // ---------------------------------------------------------------- uvw
 
+// fp32 mixing runs on the tensor cores when every block has at most 256 channels.
+bool use_tc(const Plan& P) {
+  if (P.dtype != TP_F32) return false;
+  for (auto& b : P.bout) if (b.mul > 256) return false;
+  for (auto& b : P.bin) if (b.mul > 256) return false;
+  return true;
+}
+
 template <typename T>
 cudaError_t sbuild(const Plan& P, const UvwSParams<T>& p, int dir, cudaStream_t s) {
-  return P.KP == 8 ? launch_uvw_sbuild<T, 8>(p, dir, s) : launch_uvw_sbuild<T, 16>(p, dir, s);
+  if (dir == 0) return P.KP == 8 ? launch_uvw_sbuild_dir<T, 8, 0>(p, s) : launch_uvw_sbuild_dir<T, 16, 0>(p, s);
+  return P.KP == 8 ? launch_uvw_sbuild_dir<T, 8, 1>(p, s) : launch_uvw_sbuild_dir<T, 16, 1>(p, s);
 }
 
 template <typename T>
@@ -160,10 +169,12 @@ void fill_blocks(UvwSParams<T>& p, const std::vector<UvwBlockD>& blocks, const s
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
 // m_g = S_g B_g for every output block of one receiver chunk (rows -> out).
+// fp32 runs on the tensor cores (3xTF32, Bf holds the transposed operand Bt);
+// fp64 runs the SIMT GEMM (Bf holds B).
 template <typename T>
 cudaError_t mix_out(const Plan& P, const T* S, const T* Bf, T* out, int r0, int nr, int nr_alloc,
                     const std::vector<UvwBlockD>& blocks, const std::vector<long long>& b_off, long long ld_out,
-                    cudaStream_t s) {
+                    int* err, cudaStream_t s) {
   GemmBatch<T> gb;
   int n = 0, mm = 0, mn = 0;
   for (size_t g = 0; g < blocks.size(); ++g) {
@@ -179,7 +190,11 @@ cudaError_t mix_out(const Plan& P, const T* S, const T* Bf, T* out, int r0, int 
     mm = std::max(mm, q.M);
     mn = std::max(mn, q.N);
     if (n == kMaxGemmBatch || g + 1 == blocks.size()) {
-      cudaError_t e = launch_gemm<T>(0, gb, n, mm, mn, s);
+      cudaError_t e;
+      if constexpr (std::is_same<T, float>::value)
+        e = use_tc(P) ? launch_gemm_tc(gb, n, mm, err, s) : launch_gemm<T>(0, gb, n, mm, mn, s);
+      else
+        e = launch_gemm<T>(0, gb, n, mm, mn, s);
       if (e != cudaSuccess) return e;
       n = mm = mn = 0;
     }
@@ -193,7 +208,8 @@ int forward_uvw(const Plan& P, const void* x, const void* Y, const void* phi, co
   const size_t b = sizeof(T);
   T* Bf = (T*)ws;
   T* S = (T*)((char*)ws + align256((size_t)P.K * P.n_w * b));
-  cudaError_t e = launch_pack_a<T>(P.pack, (const T*)A, Bf, nullptr, s);
+  const bool tc = use_tc(P);
+  cudaError_t e = launch_pack_a<T>(P.pack, (const T*)A, tc ? nullptr : Bf, nullptr, tc ? Bf : nullptr, nullptr, s);
   if (e != cudaSuccess) return cuda_fail(e, "pack A");
   std::vector<long long> bf_off;
   {
@@ -214,7 +230,7 @@ int forward_uvw(const Plan& P, const void* x, const void* Y, const void* phi, co
     sp.r0 = r0;
     sp.nr = std::min(NR, N - r0);
     if ((e = sbuild<T>(P, sp, 0, s)) != cudaSuccess) return cuda_fail(e, "uvw state build");
-    if ((e = mix_out<T>(P, S, Bf, (T*)out, r0, sp.nr, NR, P.uvw_out, bf_off, P.c_out, s)) != cudaSuccess)
+    if ((e = mix_out<T>(P, S, Bf, (T*)out, r0, sp.nr, NR, P.uvw_out, bf_off, P.c_out, err, s)) != cudaSuccess)
       return cuda_fail(e, "uvw mixing");
   }
   return TP_OK;
@@ -233,7 +249,8 @@ int backward_uvw(const Plan& P, const void* x, const void* Y, const void* phi, c
   const size_t s0 = align256((size_t)NR * P.s_row_elems * b), s1 = align256((size_t)NS * P.sa_row_elems * b);
   T* S = (T*)((char*)ws + 3 * a);
   T* Sb = (T*)((char*)ws + 3 * a + std::max(s0, s1));
-  cudaError_t e = launch_pack_a<T>(P.pack, (const T*)A, Bf, Ba, s);
+  const bool tc = use_tc(P);
+  cudaError_t e = launch_pack_a<T>(P.pack, (const T*)A, Bf, tc ? nullptr : Ba, nullptr, tc ? Ba : nullptr, s);
   if (e != cudaSuccess) return cuda_fail(e, "pack A");
   std::vector<long long> bf_off, ba_off;
   {
@@ -311,7 +328,7 @@ int backward_uvw(const Plan& P, const void* x, const void* Y, const void* phi, c
     ap.r0 = s0r;
     ap.nr = std::min(NS, N - s0r);
     if ((e = sbuild<T>(P, ap, 1, s)) != cudaSuccess) return cuda_fail(e, "uvw source state build");
-    if ((e = mix_out<T>(P, S, Ba, (T*)gx, s0r, ap.nr, NS, P.uvw_in, ba_off, P.c_in, s)) != cudaSuccess)
+    if ((e = mix_out<T>(P, S, Ba, (T*)gx, s0r, ap.nr, NS, P.uvw_in, ba_off, P.c_in, err, s)) != cudaSuccess)
       return cuda_fail(e, "uvw grad_x mixing");
   }
   e = launch_unpack_a<T>(P.pack, Ab, (T*)gA, s);
@@ -547,6 +564,7 @@ int tp_get_device_error(void* stream) {
   }
   if (v & kErrIndex) return fail(TP_EDEVICE_INDEX, "a kernel met an index outside its range");
   if (v & kErrCsr) return fail(TP_EDEVICE_CSR, "a kernel met a bad row pointer");
+  if (v & kErrTimeout) return fail(TP_EDEVICE_TIMEOUT, "a kernel's bounded wait expired");
   return TP_OK;
 }
 
@@ -559,6 +577,7 @@ const char* tp_status_string(int status) {
     case TP_EWORKSPACE: return "workspace too small";
     case TP_EDEVICE_INDEX: return "device: index out of range";
     case TP_EDEVICE_CSR: return "device: bad row pointer";
+    case TP_EDEVICE_TIMEOUT: return "device: bounded wait expired";
     default: return "unknown status";
   }
 }

@@ -45,7 +45,7 @@ struct TileD {          // one channel tile of one irrep block
 };
 
 // Device error word bits (read back by tp_get_device_error).
-enum : int { kErrIndex = 1, kErrCsr = 2 };
+enum : int { kErrIndex = 1, kErrCsr = 2, kErrTimeout = 4 };
 
 template <typename T>
 struct UvuFwdParams {
@@ -122,6 +122,7 @@ struct UvwEdgeParams {        // backward: edge-owned grad_phi, grad_Y from S_ba
 
 struct PackPath {       // where the A columns of one path go in the packed GEMM operands
   int w_off, mi, mo, colf, cola;
+  int dcf, dca;         // state columns of the path's output block / input block
   long long bf_off, ba_off;
 };
 

@@ -20,14 +20,14 @@ cudaError_t launch_uvu_src(const UvuSrcParams<T>& p, int prof, cudaStream_t s);
 template <typename T>
 cudaError_t launch_reduce_slots(const T* part, T* out, int n_slots, long long n, cudaStream_t s);
 
-template <typename T, int KP>
-cudaError_t launch_uvw_sbuild(const UvwSParams<T>& p, int dir, cudaStream_t s);
+template <typename T, int KP, int DIR>
+cudaError_t launch_uvw_sbuild_dir(const UvwSParams<T>& p, cudaStream_t s);
 
 template <typename T, int KP>
 cudaError_t launch_uvw_edge(const UvwEdgeParams<T>& p, cudaStream_t s);
 
 template <typename T>
-cudaError_t launch_pack_a(const UvwPackParams& p, const T* A, T* Bf, T* Ba, cudaStream_t s);
+cudaError_t launch_pack_a(const UvwPackParams& p, const T* A, T* Bf, T* Ba, T* Btf, T* Bta, cudaStream_t s);
 
 template <typename T>
 cudaError_t launch_unpack_a(const UvwPackParams& p, const T* Bf, T* A, cudaStream_t s);
@@ -35,6 +35,9 @@ cudaError_t launch_unpack_a(const UvwPackParams& p, const T* Bf, T* A, cudaStrea
 // op 0: C = X B (C row-blocked); op 1: C = G B^T (dense); op 2: C (+)= X^T G (dense)
 template <typename T>
 cudaError_t launch_gemm(int op, const GemmBatch<T>& gb, int n_prob, int max_m, int max_n, cudaStream_t s);
+
+// op 0 on tensor cores (fp32, 3xTF32): C = X Bt^T with Bt [N, D] row-major, N <= 256
+cudaError_t launch_gemm_tc(const GemmBatch<float>& gb, int n_prob, int max_m, int* err, cudaStream_t s);
 
 size_t csr_workspace_bytes(long long n_nodes);
 cudaError_t csr_build(int N, int E, const int* src, const int* dst, int* rowptr, int* senders, int* perm,

@@ -301,6 +301,7 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
       }
       b.pend = (int)P.paths_fwd.size();
       b.dcols = cols;
+      for (int pi : by_out[g]) P.pack.paths[pi].dcf = cols;
       b.s_off = s_off;
       b.out_off = P.bout[g].offset;
       b.mul_own = P.bout[g].mul;
@@ -333,6 +334,7 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
       }
       b.pend = (int)P.paths_adj.size();
       b.dcols = cols;
+      for (int pi : by_in[b1]) P.pack.paths[pi].dca = cols;
       b.s_off = sa_off;
       b.out_off = P.bin[b1].offset;
       b.mul_own = P.bin[b1].mul;

@@ -24,8 +24,6 @@
 namespace tpc {
 namespace {
 
-constexpr int kDY = (kLmax + 1) * (kLmax + 1);
-
 // ---------------------------------------------------------------- edge pass
 //
 // One lane owns one edge: a warp takes 32 consecutive CSR edges (of any

@@ -285,9 +285,13 @@ __global__ void __launch_bounds__(kThreads) uvw_edge_kernel(const __grid_constan
 // Column (within A's row q) to packed row/col: every element of A [K, N_w] is
 // copied to the forward layout B_g [(pi, q, u), w] and the adjoint layout
 // B'_b [(pi, q, w), u] (or the reverse for the unpack of A_bar).
+// Layouts: Bf (forward, SIMT) [(pi,q,u), w]; Ba (adjoint, SIMT) [(pi,q,w), u];
+// Btf / Bta: the same transposed, [w, (pi,q,u)] / [u, (pi,q,w)] (K-major operands
+// of the tensor-core GEMM). Any output may be NULL.
 template <typename T>
 __global__ void pack_a_kernel(const __grid_constant__ UvwPackParams p, const T* __restrict__ A,
-                              T* __restrict__ Bf, T* __restrict__ Ba) {
+                              T* __restrict__ Bf, T* __restrict__ Ba, T* __restrict__ Btf,
+                              T* __restrict__ Bta) {
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (long long)p.K * p.n_w) return;
   const int q = (int)(idx / p.n_w);
@@ -302,6 +306,8 @@ __global__ void pack_a_kernel(const __grid_constant__ UvwPackParams p, const T* 
   const T v = A[idx];
   if (Bf) Bf[pp.bf_off + ((size_t)pp.colf + (size_t)q * pp.mi + u) * pp.mo + w] = v;
   if (Ba) Ba[pp.ba_off + ((size_t)pp.cola + (size_t)q * pp.mo + w) * pp.mi + u] = v;
+  if (Btf) Btf[pp.bf_off + (size_t)w * pp.dcf + pp.colf + (size_t)q * pp.mi + u] = v;
+  if (Bta) Bta[pp.ba_off + (size_t)u * pp.dca + pp.cola + (size_t)q * pp.mo + w] = v;
 }
 
 template <typename T>
@@ -323,21 +329,15 @@ __global__ void unpack_a_kernel(const __grid_constant__ UvwPackParams p, const T
 
 }  // namespace
 
-template <typename T, int KP>
-cudaError_t launch_uvw_sbuild(const UvwSParams<T>& p, int dir, cudaStream_t s) {
+template <typename T, int KP, int DIR>
+cudaError_t launch_uvw_sbuild_dir(const UvwSParams<T>& p, cudaStream_t s) {
   if (p.nr <= 0 || p.n_blocks == 0) return cudaSuccess;
   const size_t smem = sizeof(T) * (size_t)(kChunk * (2 * kLmax + 1) * 32 + kChunk * KP);
   dim3 grid(p.nr, p.n_blocks);
-  cudaError_t e;
-  if (dir == 0) {
-    auto k = uvw_sbuild_kernel<T, KP, 0>;
-    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
-    k<<<grid, kThreads, smem, s>>>(p);
-  } else {
-    auto k = uvw_sbuild_kernel<T, KP, 1>;
-    if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
-    k<<<grid, kThreads, smem, s>>>(p);
-  }
+  auto k = uvw_sbuild_kernel<T, KP, DIR>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<grid, kThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -353,10 +353,10 @@ cudaError_t launch_uvw_edge(const UvwEdgeParams<T>& p, cudaStream_t s) {
 }
 
 template <typename T>
-cudaError_t launch_pack_a(const UvwPackParams& p, const T* A, T* Bf, T* Ba, cudaStream_t s) {
+cudaError_t launch_pack_a(const UvwPackParams& p, const T* A, T* Bf, T* Ba, T* Btf, T* Bta, cudaStream_t s) {
   const long long n = (long long)p.K * p.n_w;
   if (n == 0) return cudaSuccess;
-  pack_a_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p, A, Bf, Ba);
+  pack_a_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p, A, Bf, Ba, Btf, Bta);
   return cudaGetLastError();
 }
 
@@ -368,25 +368,48 @@ cudaError_t launch_unpack_a(const UvwPackParams& p, const T* Bf, T* A, cudaStrea
   return cudaGetLastError();
 }
 
-#define TPC_INST(T, KP)                                                                    \
-  template cudaError_t launch_uvw_sbuild<T, KP>(const UvwSParams<T>&, int, cudaStream_t); \
-  template cudaError_t launch_uvw_edge<T, KP>(const UvwEdgeParams<T>&, cudaStream_t);
+#define TPC_INST_S(T, KP, DIR) \
+  template cudaError_t launch_uvw_sbuild_dir<T, KP, DIR>(const UvwSParams<T>&, cudaStream_t);
+#define TPC_INST_E(T, KP) template cudaError_t launch_uvw_edge<T, KP>(const UvwEdgeParams<T>&, cudaStream_t);
 #if TPC_WANT(0)
-TPC_INST(float, 8)
-template cudaError_t launch_pack_a<float>(const UvwPackParams&, const float*, float*, float*, cudaStream_t);
+template cudaError_t launch_pack_a<float>(const UvwPackParams&, const float*, float*, float*, float*, float*,
+                                          cudaStream_t);
 template cudaError_t launch_unpack_a<float>(const UvwPackParams&, const float*, float*, cudaStream_t);
-template cudaError_t launch_pack_a<double>(const UvwPackParams&, const double*, double*, double*, cudaStream_t);
+template cudaError_t launch_pack_a<double>(const UvwPackParams&, const double*, double*, double*, double*,
+                                           double*, cudaStream_t);
 template cudaError_t launch_unpack_a<double>(const UvwPackParams&, const double*, double*, cudaStream_t);
+TPC_INST_S(float, 8, 0)
 #endif
 #if TPC_WANT(1)
-TPC_INST(float, 16)
+TPC_INST_S(float, 8, 1)
 #endif
 #if TPC_WANT(2)
-TPC_INST(double, 8)
+TPC_INST_E(float, 8)
 #endif
 #if TPC_WANT(3)
-TPC_INST(double, 16)
+TPC_INST_S(float, 16, 0)
 #endif
-#undef TPC_INST
+#if TPC_WANT(4)
+TPC_INST_S(float, 16, 1)
+#endif
+#if TPC_WANT(5)
+TPC_INST_E(float, 16)
+#endif
+#if TPC_WANT(6)
+TPC_INST_S(double, 8, 0)
+TPC_INST_S(double, 8, 1)
+#endif
+#if TPC_WANT(7)
+TPC_INST_E(double, 8)
+#endif
+#if TPC_WANT(8)
+TPC_INST_S(double, 16, 0)
+TPC_INST_S(double, 16, 1)
+#endif
+#if TPC_WANT(9)
+TPC_INST_E(double, 16)
+#endif
+#undef TPC_INST_S
+#undef TPC_INST_E
 
 }  // namespace tpc

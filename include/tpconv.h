@@ -69,7 +69,8 @@ enum tp_status {
   TP_ECUDA = -3,          /* a CUDA runtime call failed */
   TP_EWORKSPACE = -4,     /* workspace smaller than tp_conv_workspace_size */
   TP_EDEVICE_INDEX = -5,  /* a kernel met an index outside its range */
-  TP_EDEVICE_CSR = -6     /* a kernel met a non-monotone or out-of-range row pointer */
+  TP_EDEVICE_CSR = -6,    /* a kernel met a non-monotone or out-of-range row pointer */
+  TP_EDEVICE_TIMEOUT = -7 /* a kernel's bounded wait on its tensor-core work expired */
 };
 
 typedef struct {
@@ -214,7 +215,7 @@ int tp_conv_backward_noalloc(tp_plan_t plan, const void* x, const void* Y, const
 
 /* Synchronise `stream`, then read and clear the device error word of the
  * current device. Returns TP_OK, TP_EDEVICE_INDEX, TP_EDEVICE_CSR or
- * TP_ECUDA. */
+ * TP_EDEVICE_TIMEOUT or TP_ECUDA. */
 int tp_get_device_error(void* stream);
 
 /* Static description of a status code. */
