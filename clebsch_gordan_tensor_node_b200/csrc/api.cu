@@ -143,13 +143,7 @@ int backward_uvu(const Plan& P, const void* x, const void* Y, const void* phi, c
 
 // ---------------------------------------------------------------- uvw
 
-// fp32 mixing runs on the tensor cores when every block has at most 256 channels.
-bool use_tc(const Plan& P) {
-  if (P.dtype != TP_F32) return false;
-  for (auto& b : P.bout) if (b.mul > 256) return false;
-  for (auto& b : P.bin) if (b.mul > 256) return false;
-  return true;
-}
+bool use_tc(const Plan& P) { return P.uvw_tc; }
 
 template <typename T>
 cudaError_t sbuild(const Plan& P, const UvwSParams<T>& p, int dir, cudaStream_t s) {
@@ -169,12 +163,44 @@ void fill_blocks(UvwSParams<T>& p, const std::vector<UvwBlockD>& blocks, const s
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
 // m_g = S_g B_g for every output block of one receiver chunk (rows -> out).
-// fp32 runs on the tensor cores (3xTF32, Bf holds the transposed operand Bt);
-// fp64 runs the SIMT GEMM (Bf holds B).
+// Tensor-core plans: Bf holds Bt_hi and Blo Bt_lo (transposed, split); the
+// SIMT GEMM reads Bf as B [D, N].
 template <typename T>
-cudaError_t mix_out(const Plan& P, const T* S, const T* Bf, T* out, int r0, int nr, int nr_alloc,
+cudaError_t mix_out(const Plan& P, const T* S, const T* Bf, const T* Blo, T* out, int r0, int nr, int nr_alloc,
                     const std::vector<UvwBlockD>& blocks, const std::vector<long long>& b_off, long long ld_out,
                     int* err, cudaStream_t s) {
+  if constexpr (std::is_same<T, float>::value) {
+    if (use_tc(P)) {
+      TcBatch tb;
+      int n = 0, mm = 0, npmax = 16;
+      for (size_t g = 0; g < blocks.size(); ++g) {
+        const UvwBlockD& b = blocks[g];
+        const int dc = 2 * b.l + 1, M = nr * dc, N = b.mul_own, D = b.dcols;
+        if (M == 0) continue;
+        TcProb& q = tb.prob[n];
+        const int np = (N + 15) / 16 * 16;
+        const float* X = S + (size_t)nr_alloc * b.s_off;
+        if (D > 0) {
+          if (!tc_make_map(&q.tx, X, M, D, 128) || !tc_make_map(&q.tbh, Bf + b_off[g], N, D, np) ||
+              !tc_make_map(&q.tbl, Blo + b_off[g], N, D, np))
+            return cudaErrorInvalidValue;
+        }
+        q.C = out;
+        q.c = RowBlocked{r0, dc, ld_out, b.out_off, N};
+        q.M = M; q.N = N; q.D = D; q.pad = 0;
+        ++n;
+        mm = std::max(mm, M);
+        npmax = std::max(npmax, np);
+        if (n == kMaxGemmBatch) {
+          cudaError_t e = launch_gemm_tc(tb, n, mm, npmax, err, s);
+          if (e != cudaSuccess) return e;
+          n = mm = 0;
+          npmax = 16;
+        }
+      }
+      return launch_gemm_tc(tb, n, mm, npmax, err, s);
+    }
+  }
   GemmBatch<T> gb;
   int n = 0, mm = 0, mn = 0;
   for (size_t g = 0; g < blocks.size(); ++g) {
@@ -190,11 +216,7 @@ cudaError_t mix_out(const Plan& P, const T* S, const T* Bf, T* out, int r0, int 
     mm = std::max(mm, q.M);
     mn = std::max(mn, q.N);
     if (n == kMaxGemmBatch || g + 1 == blocks.size()) {
-      cudaError_t e;
-      if constexpr (std::is_same<T, float>::value)
-        e = use_tc(P) ? launch_gemm_tc(gb, n, mm, err, s) : launch_gemm<T>(0, gb, n, mm, mn, s);
-      else
-        e = launch_gemm<T>(0, gb, n, mm, mn, s);
+      cudaError_t e = launch_gemm<T>(0, gb, n, mm, mn, s);
       if (e != cudaSuccess) return e;
       n = mm = mn = 0;
     }
@@ -206,10 +228,13 @@ template <typename T>
 int forward_uvw(const Plan& P, const void* x, const void* Y, const void* phi, const void* A, const int* rowptr,
                 const int* senders, int N, int E, void* out, void* ws, int* err, cudaStream_t s) {
   const size_t b = sizeof(T);
-  T* Bf = (T*)ws;
-  T* S = (T*)((char*)ws + align256((size_t)P.K * P.n_w * b));
   const bool tc = use_tc(P);
-  cudaError_t e = launch_pack_a<T>(P.pack, (const T*)A, tc ? nullptr : Bf, nullptr, tc ? Bf : nullptr, nullptr, s);
+  const size_t a = align256((size_t)P.K * P.n_w * b);
+  T* Bf = (T*)ws;
+  T* Blo = tc ? (T*)((char*)ws + a) : nullptr;
+  T* S = (T*)((char*)ws + (tc ? 2 : 1) * a);
+  cudaError_t e = launch_pack_a<T>(P.pack, (const T*)A, tc ? nullptr : Bf, nullptr, tc ? Bf : nullptr, nullptr,
+                                   Blo, nullptr, s);
   if (e != cudaSuccess) return cuda_fail(e, "pack A");
   std::vector<long long> bf_off;
   {
@@ -230,7 +255,7 @@ int forward_uvw(const Plan& P, const void* x, const void* Y, const void* phi, co
     sp.r0 = r0;
     sp.nr = std::min(NR, N - r0);
     if ((e = sbuild<T>(P, sp, 0, s)) != cudaSuccess) return cuda_fail(e, "uvw state build");
-    if ((e = mix_out<T>(P, S, Bf, (T*)out, r0, sp.nr, NR, P.uvw_out, bf_off, P.c_out, err, s)) != cudaSuccess)
+    if ((e = mix_out<T>(P, S, Bf, Blo, (T*)out, r0, sp.nr, NR, P.uvw_out, bf_off, P.c_out, err, s)) != cudaSuccess)
       return cuda_fail(e, "uvw mixing");
   }
   return TP_OK;
@@ -242,15 +267,18 @@ int backward_uvw(const Plan& P, const void* x, const void* Y, const void* phi, c
                  int N, int E, void* gx, void* gY, void* gphi, void* gA, void* ws, int* err, cudaStream_t s) {
   const size_t b = sizeof(T);
   const size_t a = align256((size_t)P.K * P.n_w * b);
+  const bool tc = use_tc(P);
   T* Bf = (T*)ws;
   T* Ba = (T*)((char*)ws + a);
   T* Ab = (T*)((char*)ws + 2 * a);
+  T* Balo = tc ? (T*)((char*)ws + 3 * a) : nullptr;
+  const size_t na = tc ? 4 : 3;
   const int NR = uvw_chunk_rows(P, N, 0), NS = uvw_chunk_rows(P, N, 1);
   const size_t s0 = align256((size_t)NR * P.s_row_elems * b), s1 = align256((size_t)NS * P.sa_row_elems * b);
-  T* S = (T*)((char*)ws + 3 * a);
-  T* Sb = (T*)((char*)ws + 3 * a + std::max(s0, s1));
-  const bool tc = use_tc(P);
-  cudaError_t e = launch_pack_a<T>(P.pack, (const T*)A, Bf, tc ? nullptr : Ba, nullptr, tc ? Ba : nullptr, s);
+  T* S = (T*)((char*)ws + na * a);
+  T* Sb = (T*)((char*)ws + na * a + std::max(s0, s1));
+  cudaError_t e = launch_pack_a<T>(P.pack, (const T*)A, Bf, tc ? nullptr : Ba, nullptr, tc ? Ba : nullptr, nullptr,
+                                   Balo, s);
   if (e != cudaSuccess) return cuda_fail(e, "pack A");
   std::vector<long long> bf_off, ba_off;
   {
@@ -328,7 +356,7 @@ int backward_uvw(const Plan& P, const void* x, const void* Y, const void* phi, c
     ap.r0 = s0r;
     ap.nr = std::min(NS, N - s0r);
     if ((e = sbuild<T>(P, ap, 1, s)) != cudaSuccess) return cuda_fail(e, "uvw source state build");
-    if ((e = mix_out<T>(P, S, Ba, (T*)gx, s0r, ap.nr, NS, P.uvw_in, ba_off, P.c_in, err, s)) != cudaSuccess)
+    if ((e = mix_out<T>(P, S, Ba, Balo, (T*)gx, s0r, ap.nr, NS, P.uvw_in, ba_off, P.c_in, err, s)) != cudaSuccess)
       return cuda_fail(e, "uvw grad_x mixing");
   }
   e = launch_unpack_a<T>(P.pack, Ab, (T*)gA, s);

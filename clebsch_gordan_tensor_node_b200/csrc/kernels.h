@@ -1,6 +1,7 @@
 // Launchers of the tensor-product convolution kernels (internal to the library).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -26,8 +27,11 @@ cudaError_t launch_uvw_sbuild_dir(const UvwSParams<T>& p, cudaStream_t s);
 template <typename T, int KP>
 cudaError_t launch_uvw_edge(const UvwEdgeParams<T>& p, cudaStream_t s);
 
+// Bf, Ba: SIMT operand layouts; Btf / Bta: transposed (K-major) operands, holding
+// the TF32-exact high parts when Btf_lo / Bta_lo are given (which get the rest).
 template <typename T>
-cudaError_t launch_pack_a(const UvwPackParams& p, const T* A, T* Bf, T* Ba, T* Btf, T* Bta, cudaStream_t s);
+cudaError_t launch_pack_a(const UvwPackParams& p, const T* A, T* Bf, T* Ba, T* Btf, T* Bta, T* Btf_lo,
+                          T* Bta_lo, cudaStream_t s);
 
 template <typename T>
 cudaError_t launch_unpack_a(const UvwPackParams& p, const T* Bf, T* A, cudaStream_t s);
@@ -36,8 +40,20 @@ cudaError_t launch_unpack_a(const UvwPackParams& p, const T* Bf, T* A, cudaStrea
 template <typename T>
 cudaError_t launch_gemm(int op, const GemmBatch<T>& gb, int n_prob, int max_m, int max_n, cudaStream_t s);
 
-// op 0 on tensor cores (fp32, 3xTF32): C = X Bt^T with Bt [N, D] row-major, N <= 256
-cudaError_t launch_gemm_tc(const GemmBatch<float>& gb, int n_prob, int max_m, int* err, cudaStream_t s);
+// op 0 on tensor cores (fp32, 3xTF32): C = X Bt^T with X [M, D] and Bt [N, D]
+// row-major, read through TMA tensor maps (box 32 x 128 for X, 32 x N16 for Bt).
+struct TcProb {
+  CUtensorMap tx, tbh, tbl;   // X (raw), Bt_hi, Bt_lo
+  float* C;
+  RowBlocked c;
+  int M, N, D, pad;
+};
+struct TcBatch {
+  TcProb prob[kMaxGemmBatch];
+};
+bool tc_gemm_available();
+bool tc_make_map(CUtensorMap* map, const float* base, long long rows, long long cols, int box_rows);
+cudaError_t launch_gemm_tc(const TcBatch& tb, int n_prob, int max_m, int npmax, int* err, cudaStream_t s);
 
 size_t csr_workspace_bytes(long long n_nodes);
 cudaError_t csr_build(int N, int E, const int* src, const int* dst, int* rowptr, int* senders, int* perm,

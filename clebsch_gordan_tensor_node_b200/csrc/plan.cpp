@@ -343,6 +343,12 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
       P.uvw_in.push_back(b);
     }
     P.sa_row_elems = sa_off;
+    // tensor-core mixing: fp32, at most 64 channels per block (one 128 x 64 tile
+    // pipeline fits shared memory), state rows whose width is a multiple of 4
+    // (16-byte TMA strides)
+    P.uvw_tc = dtype == TP_F32;
+    for (auto& b : P.uvw_out) P.uvw_tc = P.uvw_tc && b.mul_own <= 64 && b.dcols % 4 == 0;
+    for (auto& b : P.uvw_in) P.uvw_tc = P.uvw_tc && b.mul_own <= 64 && b.dcols % 4 == 0;
     const size_t bsz2 = dtype == TP_F32 ? 4 : 8;
     if ((size_t)std::max(P.s_row_elems, P.sa_row_elems) * bsz2 > kUvwChunkBytes) {
       msg = "one node's uvw state exceeds the state chunk budget";
@@ -380,7 +386,9 @@ size_t workspace_bytes(const Plan& p, long long n_nodes, int pass) {
     const size_t a = ((size_t)p.K * p.n_w * b + 255) / 256 * 256;
     const size_t s0 = ((size_t)uvw_chunk_rows(p, n_nodes, 0) * p.s_row_elems * b + 255) / 256 * 256;
     const size_t s1 = ((size_t)uvw_chunk_rows(p, n_nodes, 1) * p.sa_row_elems * b + 255) / 256 * 256;
-    bytes = pass == 0 ? a + s0 : 3 * a + 2 * std::max(s0, s1);
+    // the tensor-core path adds the low parts of the transposed operands
+    const size_t na = pass == 0 ? (p.uvw_tc ? 2 : 1) : (p.uvw_tc ? 4 : 3);
+    bytes = na * a + (pass == 0 ? s0 : 2 * std::max(s0, s1));
   }
   return (bytes + 255) / 256 * 256;
 }

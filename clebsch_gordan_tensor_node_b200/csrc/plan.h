@@ -47,6 +47,7 @@ struct Plan {
   UvwPackParams pack{};
   long long s_row_elems = 0;        // state elements per receiver (S)
   long long sa_row_elems = 0;       // state elements per source (S')
+  bool uvw_tc = false;              // channel mixing on the tensor cores (fp32)
 };
 
 // Bytes of one uvw state chunk (the scratch budget of Sobek App. B.2).

@@ -289,9 +289,17 @@ __global__ void __launch_bounds__(kThreads) uvw_edge_kernel(const __grid_constan
 // Btf / Bta: the same transposed, [w, (pi,q,u)] / [u, (pi,q,w)] (K-major operands
 // of the tensor-core GEMM). Any output may be NULL.
 template <typename T>
+__device__ __forceinline__ T hi_part(T v) {
+  if constexpr (sizeof(T) == 4)
+    return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
+  else
+    return v;
+}
+
+template <typename T>
 __global__ void pack_a_kernel(const __grid_constant__ UvwPackParams p, const T* __restrict__ A,
                               T* __restrict__ Bf, T* __restrict__ Ba, T* __restrict__ Btf,
-                              T* __restrict__ Bta) {
+                              T* __restrict__ Bta, T* __restrict__ Btf_lo, T* __restrict__ Bta_lo) {
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (long long)p.K * p.n_w) return;
   const int q = (int)(idx / p.n_w);
@@ -306,8 +314,17 @@ __global__ void pack_a_kernel(const __grid_constant__ UvwPackParams p, const T* 
   const T v = A[idx];
   if (Bf) Bf[pp.bf_off + ((size_t)pp.colf + (size_t)q * pp.mi + u) * pp.mo + w] = v;
   if (Ba) Ba[pp.ba_off + ((size_t)pp.cola + (size_t)q * pp.mo + w) * pp.mi + u] = v;
-  if (Btf) Btf[pp.bf_off + (size_t)w * pp.dcf + pp.colf + (size_t)q * pp.mi + u] = v;
-  if (Bta) Bta[pp.ba_off + (size_t)u * pp.dca + pp.cola + (size_t)q * pp.mo + w] = v;
+  const T vh = hi_part(v);
+  if (Btf) {
+    const size_t o = pp.bf_off + (size_t)w * pp.dcf + pp.colf + (size_t)q * pp.mi + u;
+    Btf[o] = Btf_lo ? vh : v;
+    if (Btf_lo) Btf_lo[o] = v - vh;
+  }
+  if (Bta) {
+    const size_t o = pp.ba_off + (size_t)u * pp.dca + pp.cola + (size_t)q * pp.mo + w;
+    Bta[o] = Bta_lo ? vh : v;
+    if (Bta_lo) Bta_lo[o] = v - vh;
+  }
 }
 
 template <typename T>
@@ -353,10 +370,11 @@ cudaError_t launch_uvw_edge(const UvwEdgeParams<T>& p, cudaStream_t s) {
 }
 
 template <typename T>
-cudaError_t launch_pack_a(const UvwPackParams& p, const T* A, T* Bf, T* Ba, T* Btf, T* Bta, cudaStream_t s) {
+cudaError_t launch_pack_a(const UvwPackParams& p, const T* A, T* Bf, T* Ba, T* Btf, T* Bta, T* Btf_lo,
+                          T* Bta_lo, cudaStream_t s) {
   const long long n = (long long)p.K * p.n_w;
   if (n == 0) return cudaSuccess;
-  pack_a_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p, A, Bf, Ba, Btf, Bta);
+  pack_a_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p, A, Bf, Ba, Btf, Bta, Btf_lo, Bta_lo);
   return cudaGetLastError();
 }
 
@@ -373,10 +391,10 @@ cudaError_t launch_unpack_a(const UvwPackParams& p, const T* Bf, T* A, cudaStrea
 #define TPC_INST_E(T, KP) template cudaError_t launch_uvw_edge<T, KP>(const UvwEdgeParams<T>&, cudaStream_t);
 #if TPC_WANT(0)
 template cudaError_t launch_pack_a<float>(const UvwPackParams&, const float*, float*, float*, float*, float*,
-                                          cudaStream_t);
+                                          float*, float*, cudaStream_t);
 template cudaError_t launch_unpack_a<float>(const UvwPackParams&, const float*, float*, cudaStream_t);
 template cudaError_t launch_pack_a<double>(const UvwPackParams&, const double*, double*, double*, double*,
-                                           double*, cudaStream_t);
+                                           double*, double*, double*, cudaStream_t);
 template cudaError_t launch_unpack_a<double>(const UvwPackParams&, const double*, double*, cudaStream_t);
 TPC_INST_S(float, 8, 0)
 #endif
