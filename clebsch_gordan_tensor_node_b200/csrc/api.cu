@@ -277,7 +277,11 @@ int backward_uvw(const Plan& P, const void* x, const void* Y, const void* phi, c
   const size_t s0 = align256((size_t)NR * P.s_row_elems * b), s1 = align256((size_t)NS * P.sa_row_elems * b);
   T* S = (T*)((char*)ws + na * a);
   T* Sb = (T*)((char*)ws + na * a + std::max(s0, s1));
-  cudaError_t e = launch_pack_a<T>(P.pack, (const T*)A, Bf, tc ? nullptr : Ba, nullptr, tc ? Ba : nullptr, nullptr,
+  // Bf feeds only S_bar = m_bar Bf^T here: rows in (u, q) order give S_bar the
+  // column order of the edge pass
+  UvwPackParams pk = P.pack;
+  pk.bf_uq = 1;
+  cudaError_t e = launch_pack_a<T>(pk, (const T*)A, Bf, tc ? nullptr : Ba, nullptr, tc ? Ba : nullptr, nullptr,
                                    Balo, s);
   if (e != cudaSuccess) return cuda_fail(e, "pack A");
   std::vector<long long> bf_off, ba_off;
@@ -309,6 +313,28 @@ int backward_uvw(const Plan& P, const void* x, const void* Y, const void* phi, c
   std::memcpy(ep.blocks, P.uvw_out.data(), P.uvw_out.size() * sizeof(UvwBlockD));
   std::memcpy(ep.paths, P.paths_fwd.data(), P.paths_fwd.size() * sizeof(PathD));
   ep.n_blocks = (int)P.uvw_out.size();
+  {
+    const int vw = 16 / (int)b;
+    bool vec = P.K == P.KP && P.c_in % vw == 0;
+    int xs = 0, sbar = 0;
+    for (const PathD& pd : P.paths_fwd) {
+      vec = vec && pd.x_off % vw == 0 && pd.mul_in % vw == 0;
+      const int nc = std::min(kEdgeTile, pd.mul_in);
+      xs = std::max(xs, 32 * edge_slot_stride((2 * pd.l1 + 1) * nc));
+      sbar = std::max(sbar, (2 * pd.l3 + 1) * nc * P.K);
+    }
+    for (size_t g = 0; g < P.uvw_out.size(); ++g)
+      for (int pi = P.uvw_out[g].pbeg; pi < P.uvw_out[g].pend; ++pi) ep.path_blk[pi] = (int8_t)g;
+    // the phi_bar partials [warps][K][32] reuse stage buffer 0 at the end of a round
+    xs = std::max(xs, kEdgeWarps * 32 * P.K - sbar);
+    ep.vec = vec ? 1 : 0;
+    ep.smem_sbar = (int)((sbar * b + 15) / 16 * 16);
+    ep.smem_stage = (int)((xs * b + 15) / 16 * 16) + ep.smem_sbar;
+    ep.smem_red = (int)((kEdgeWarps * 32 * P.dim_y * b + 15) / 16 * 16);
+    ep.smem_ct = (int)(kEdgeWarps * 32 * (2 * kLmax + 1) * b);
+    if (2 * (size_t)ep.smem_stage + ep.smem_red + ep.smem_ct + 32 * sizeof(int) > (size_t)227 * 1024)
+      return fail(TP_EUNSUPPORTED, "uvw edge pass: staging buffers exceed 227 KiB of shared memory");
+  }
   for (int r0 = 0; r0 < N; r0 += NR) {
     const int nr = std::min(NR, N - r0);
     sp.r0 = r0;

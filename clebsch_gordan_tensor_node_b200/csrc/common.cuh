@@ -68,6 +68,7 @@ struct UvuEdgeParams {        // backward: edge-owned grad_phi, grad_Y
   T* gY; T* gphi; int* err;
   int N, E, K, c_in, c_out, dim_y, n_w;
   int n_paths;
+  int split;                  // warps that share one group of 32 edges (paths dealt round-robin)
   PathD paths[kMaxPaths];     // canonical order
 };
 
@@ -109,13 +110,25 @@ struct UvwSParams {           // S (dir 0: receivers gather x) or S' (dir 1: sou
   PathD paths[kMaxPaths];     // x_off / mul_in describe the gathered block
 };
 
+// Edge pass of the uvw backward: input channels staged per tile, warps per
+// CTA, and the per-sender row stride in the staging buffer for a tile row of n
+// scalars: odd, so that 32 lanes reading one scalar each from their own row
+// hit 32 distinct banks.
+constexpr int kEdgeTile = 16;
+constexpr int kEdgeWarps = 4, kEdgeThreads = 32 * kEdgeWarps;
+__host__ __device__ constexpr int edge_slot_stride(int n) { return n | 1; }
+
 template <typename T>
 struct UvwEdgeParams {        // backward: edge-owned grad_phi, grad_Y from S_bar
-  const T* x; const T* Y; const T* phi; const T* Sbar;
+  const T* x; const T* Y; const T* phi; const T* Sbar;   // S_bar columns per path: (u, q)
   const int* rowptr; const int* senders;
   T* gY; T* gphi; int* err;
   int N, E, K, c_in, dim_y;
   int r0, nr, nr_alloc, n_blocks;
+  int vec;                     // 16-byte copies: K == KP; c_in, x_off, mul_in multiples of 16 bytes
+  int smem_stage, smem_sbar;   // bytes of one stage buffer (x part, then S_bar part) and its S_bar part
+  int smem_red, smem_ct;       // bytes of the per-warp Y_bar region and of the C / T_bar columns
+  int8_t path_blk[kMaxPaths];  // owner block of each path
   UvwBlockD blocks[kMaxBlocks];
   PathD paths[kMaxPaths];
 };
@@ -128,6 +141,7 @@ struct PackPath {       // where the A columns of one path go in the packed GEMM
 
 struct UvwPackParams {
   int K, n_w, n_paths;
+  int bf_uq;            // rows of Bf per path in (u, q) order instead of (q, u)
   PackPath paths[kMaxPaths];
 };
 

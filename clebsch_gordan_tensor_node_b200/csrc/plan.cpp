@@ -277,6 +277,7 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
     // same (path, q, u) order
     long long s_off = 0, bf_off = 0;
     P.pack.K = P.K;
+    P.pack.bf_uq = 0;
     P.pack.n_w = (int)P.n_w;
     P.pack.n_paths = (int)P.paths.size();
     for (size_t g = 0; g < P.bout.size(); ++g) {

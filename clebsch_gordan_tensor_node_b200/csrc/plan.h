@@ -51,7 +51,7 @@ struct Plan {
 };
 
 // Bytes of one uvw state chunk (the scratch budget of Sobek App. B.2).
-constexpr size_t kUvwChunkBytes = size_t(256) << 20;
+constexpr size_t kUvwChunkBytes = size_t(1) << 30;
 // Owners per uvw state chunk for a problem of n_nodes nodes (dir 0: S, 1: S').
 int uvw_chunk_rows(const Plan& p, long long n_nodes, int dir);
 

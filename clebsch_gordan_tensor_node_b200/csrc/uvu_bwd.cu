@@ -24,6 +24,8 @@
 namespace tpc {
 namespace {
 
+constexpr long long kSplitEdgeGroups = 148LL * kWarpsPerBlock;   // 32-edge groups below which paths split
+
 // ---------------------------------------------------------------- edge pass
 //
 // One lane owns one edge: a warp takes 32 consecutive CSR edges (of any
@@ -32,6 +34,10 @@ namespace {
 // path the lane contracts its Y block with the CG pairs once (cY); the channel
 // loop then reads A as a warp-uniform 16-byte broadcast and x_j, m_bar_i as
 // per-lane 16-byte gathers, V channels at a time.
+//
+// Graphs with few edges would leave most SMs idle that way, so there all the
+// warps of a CTA share one group of 32 edges and deal the paths round-robin;
+// their partial sums are added in warp order in shared memory (split mode).
 
 template <int L1M, int L2M, int L3M>
 struct Prof {
@@ -119,9 +125,10 @@ template <typename T, int KP, int V, class PR>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 uvu_edge_kernel(const __grid_constant__ UvuEdgeParams<T> p) {
   constexpr int DY = (PR::l2 + 1) * (PR::l2 + 1);
-  const int lane = threadIdx.x & 31;
-  const long long e0 = ((long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5)) * 32;
-  if (e0 >= p.E) return;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const bool split = p.split > 1;
+  const long long e0 = split ? (long long)blockIdx.x * 32 : ((long long)blockIdx.x * kWarpsPerBlock + warp) * 32;
+  if (e0 >= p.E) return;   // uniform over the CTA in split mode
   const int e = (int)(e0 + lane);
   const bool live = e < p.E;
   // receiver of CSR position e: the last i with rowptr[i] <= e
@@ -149,7 +156,7 @@ uvu_edge_kernel(const __grid_constant__ UvuEdgeParams<T> p) {
 #pragma unroll
   for (int m = 0; m < DY; ++m) gY[m] = T(0);
   if (live) {
-    for (int pi = 0; pi < p.n_paths; ++pi) {
+    for (int pi = split ? warp : 0; pi < p.n_paths; pi += split ? p.split : 1) {
       const PathD& pd = p.paths[pi];
       dispatch_l<PR::l1>(pd.l1, [&](auto A1) {
         constexpr int L1 = decltype(A1)::value;
@@ -169,6 +176,30 @@ uvu_edge_kernel(const __grid_constant__ UvuEdgeParams<T> p) {
 #pragma unroll
       for (int m = 0; m < DY; ++m) gY[m] = T(0);
     }
+  }
+  if (split) {
+    // add the warps' partial sums in warp order: red[warp][v][lane]
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    T* red = reinterpret_cast<T*>(smem_raw);
+    const int nv = p.K + p.dim_y;
+    T* mine = red + (size_t)warp * nv * 32 + lane;
+#pragma unroll
+    for (int q = 0; q < KP; ++q)
+      if (q < p.K) mine[q * 32] = gphi[q];
+#pragma unroll
+    for (int m = 0; m < DY; ++m)
+      if (m < p.dim_y) mine[(p.K + m) * 32] = gY[m];
+    __syncthreads();
+    for (int t = threadIdx.x; t < nv * 32; t += blockDim.x) {
+      const int v = t >> 5, sl = t & 31;
+      const long long eo = e0 + sl;
+      if (eo >= p.E) continue;
+      T acc = red[(size_t)v * 32 + sl];
+      for (int w = 1; w < p.split; ++w) acc += red[((size_t)w * nv + v) * 32 + sl];
+      if (v < p.K) p.gphi[(size_t)eo * p.K + v] = acc;
+      else p.gY[(size_t)eo * p.dim_y + (v - p.K)] = acc;
+    }
+  } else if (live) {
 #pragma unroll
     for (int q = 0; q < KP; ++q)
       if (q < p.K) p.gphi[(size_t)e * p.K + q] = gphi[q];
@@ -416,18 +447,32 @@ __global__ void reduce_slots_kernel(const T* __restrict__ part, T* __restrict__ 
 
 }  // namespace
 
-template <typename T, int KP, int V>
-cudaError_t launch_uvu_edge(const UvuEdgeParams<T>& p, int prof, cudaStream_t s) {
-  if (p.N == 0 || p.E == 0) return cudaSuccess;
-  const long long warps = ((long long)p.E + 31) / 32;
-  const unsigned blocks = (unsigned)((warps + kWarpsPerBlock - 1) / kWarpsPerBlock);
-  switch (prof) {
-    case 0: uvu_edge_kernel<T, KP, V, Prof<2, 2, 2>><<<blocks, kWarpsPerBlock * 32, 0, s>>>(p); break;
-    case 1: uvu_edge_kernel<T, KP, V, Prof<1, 3, 3>><<<blocks, kWarpsPerBlock * 32, 0, s>>>(p); break;
-    case 2: uvu_edge_kernel<T, KP, V, Prof<3, 3, 3>><<<blocks, kWarpsPerBlock * 32, 0, s>>>(p); break;
-    default: uvu_edge_kernel<T, KP, V, Prof<4, 4, 4>><<<blocks, kWarpsPerBlock * 32, 0, s>>>(p); break;
+template <typename T, int KP, int V, class PR>
+cudaError_t launch_edge_prof(const UvuEdgeParams<T>& p, unsigned blocks, size_t smem, cudaStream_t s) {
+  auto kern = uvu_edge_kernel<T, KP, V, PR>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
   }
+  kern<<<blocks, kWarpsPerBlock * 32, smem, s>>>(p);
   return cudaGetLastError();
+}
+
+template <typename T, int KP, int V>
+cudaError_t launch_uvu_edge(const UvuEdgeParams<T>& p0, int prof, cudaStream_t s) {
+  if (p0.N == 0 || p0.E == 0) return cudaSuccess;
+  UvuEdgeParams<T> p = p0;
+  const long long groups = ((long long)p.E + 31) / 32;
+  // split mode while one warp per 32 edges would give fewer than 8 warps per SM
+  p.split = groups < kSplitEdgeGroups ? kWarpsPerBlock : 1;
+  const unsigned blocks = (unsigned)(p.split > 1 ? groups : (groups + kWarpsPerBlock - 1) / kWarpsPerBlock);
+  const size_t smem = p.split > 1 ? sizeof(T) * (size_t)kWarpsPerBlock * (p.K + p.dim_y) * 32 : 0;
+  switch (prof) {
+    case 0: return launch_edge_prof<T, KP, V, Prof<2, 2, 2>>(p, blocks, smem, s);
+    case 1: return launch_edge_prof<T, KP, V, Prof<1, 3, 3>>(p, blocks, smem, s);
+    case 2: return launch_edge_prof<T, KP, V, Prof<3, 3, 3>>(p, blocks, smem, s);
+    default: return launch_edge_prof<T, KP, V, Prof<4, 4, 4>>(p, blocks, smem, s);
+  }
 }
 
 template <typename T, int KP, int CPL, class PR>

@@ -145,138 +145,269 @@ __global__ void __launch_bounds__(kThreads) uvw_sbuild_kernel(const __grid_const
 }
 
 // ---------------------------------------------------------------- edge pass
+//
+// One CTA (kEdgeWarps warps) per receiver r. The receiver's edges go in rounds
+// of 32: lane l of every warp owns edge slot l of the round. The work of a
+// round is a sequence of stages, one per (path, tile of kEdgeTile input
+// channels u); each warp takes an equal share of the tile's channels. For each
+// stage the CTA copies into shared memory the gathered x[m1][u] of the 32
+// senders and S_bar[mo][u][q] of r, with cp.async, one stage ahead of the
+// arithmetic (two buffers). S_bar of r is laid out per path as (mo, u, q) with
+// the K radial values contiguous (the backward packs A in that column order),
+// so all lanes of a warp read the same S_bar values (shared-memory broadcast)
+// while each contracts its own edge:
+//   C[mo]        = sum c x[mi] Y[my]                     (per edge, channel u)
+//   T_bar[u][mo] = sum_q phi_e[q] S_bar[mo][u][q]
+//   phi_bar_e[q] += sum_{u,mo} S_bar[mo][u][q] C[mo]
+//   Y_bar_e[my]  += sum c x[mi] T_bar[mo]
+// The loops over u and mo are not unrolled (C and T_bar pass through a
+// per-lane shared column), which keeps a path's loop body small enough for the
+// instruction cache. phi_bar_e accumulates in registers, Y_bar_e in a per-warp
+// shared column; the warps' partial sums are added in warp order at the end of
+// the round, so the result does not depend on timing.
 
-constexpr int kEdgeChunk = 64;
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src) : "memory");
+}
+template <int B>
+__device__ __forceinline__ void cp_async_small(void* dst, const void* src) {   // B = 4 or 8 bytes
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], %2;\n" ::"r"(d), "l"(src), "n"(B) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
+struct EdgeStage {
+  int pi, c0;   // path and first channel of the tile; pi == n_paths ends the round
+};
+
+// Issue the copies of one stage into buffer (Xs, Ss). x goes as single
+// scalars into [slot][mi][u] rows of odd stride (conflict-free reads by slot);
+// S_bar as 16-byte pieces where the layout allows, else plain loads.
 template <typename T>
-__device__ __forceinline__ T wsum(T v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
+__device__ __forceinline__ void edge_stage_issue(const UvwEdgeParams<T>& p, const EdgeStage& st, int r,
+                                                 const int* js, T* Xs, T* Ss) {
+  constexpr int VW = sizeof(T) == 4 ? 4 : 2;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const PathD& pd = p.paths[st.pi];
+  const UvwBlockD& bd = p.blocks[p.path_blk[st.pi]];
+  const int d1 = 2 * pd.l1 + 1, d3 = 2 * pd.l3 + 1, mi = pd.mul_in;
+  const int nc = min(kEdgeTile, mi - st.c0), row = d1 * nc, ss = edge_slot_stride(row);
+  const T* xb = p.x + pd.x_off + st.c0;
+  const T* sb = p.Sbar + (size_t)p.nr_alloc * bd.s_off + (size_t)(r - p.r0) * d3 * bd.dcols + pd.col_off +
+                (size_t)st.c0 * p.K;
+  const int srow = nc * p.K;   // S_bar scalars per component in the tile
+  for (int sl = warp; sl < 32; sl += kEdgeWarps) {
+    const T* src = xb + (size_t)js[sl] * p.c_in;
+    T* dst = Xs + sl * ss;
+    for (int c = lane; c < row; c += 32) {
+      const int m = c / nc, u = c - m * nc;
+      if (p.vec)
+        cp_async_small<sizeof(T)>(dst + c, src + m * mi + u);
+      else
+        dst[c] = ldg(src + m * mi + u);
+    }
+  }
+  if (p.vec) {
+    const int nsv = srow / VW;
+    for (int t = threadIdx.x; t < d3 * nsv; t += kEdgeThreads) {
+      const int m = t / nsv, c = (t - m * nsv) * VW;
+      cp_async16(Ss + m * srow + c, sb + (size_t)m * bd.dcols + c);
+    }
+  } else {
+    for (int t = threadIdx.x; t < d3 * srow; t += kEdgeThreads) {
+      const int m = t / srow, c = t - m * srow;
+      Ss[m * srow + c] = ldg(sb + (size_t)m * bd.dcols + c);
+    }
+  }
 }
 
-template <typename T, int KP, int L1, int L2, int L3>
-__device__ __forceinline__ void edge_path(const UvwEdgeParams<T>& p, const UvwBlockD& bd, const PathD& pd,
-                                          int r, int ec, int n, T* Sb, T* acc) {
+template <typename T, int L1, int L2, int L3, int KP>
+__device__ __forceinline__ void edge_stage_compute(const UvwEdgeParams<T>& p, const PathD& pd, int c0, int e,
+                                                   bool ok, const T* Xs, const T* Ss, T* CT,
+                                                   const T (&ph)[KP], T (&gphi)[KP], T* gyr) {
   using CGp = cgt::CG<L1, L2, L3>;
-  constexpr int D1 = 2 * L1 + 1, D2 = 2 * L2 + 1, D3 = 2 * L3 + 1;
+  constexpr int D1 = 2 * L1 + 1, D2 = 2 * L2 + 1, D3 = 2 * L3 + 1, NP = CGp::npair, Y0 = L2 * L2;
+  constexpr int VW = sizeof(T) == 4 ? 4 : 2;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mi = pd.mul_in;
-  const int accw = p.K + p.dim_y;
-  for (int c0 = 0; c0 < mi; c0 += 32) {
-    // stage S_bar of receiver r, this path, channel tile: Sb[q][m3][lane]
-    const T* src = p.Sbar + (size_t)p.nr_alloc * bd.s_off + (size_t)(r - p.r0) * D3 * bd.dcols + pd.col_off + c0;
-    for (int t = threadIdx.x; t < KP * D3 * 32; t += kThreads) {
-      const int c = t & 31, m3 = (t >> 5) % D3, q = (t >> 5) / D3;
-      Sb[t] = (q < p.K && c0 + c < mi) ? src[(size_t)m3 * bd.dcols + (size_t)q * mi + c] : T(0);
-    }
-    __syncthreads();
-    const bool act = c0 + lane < mi;
-    const int cl = act ? c0 + lane : c0;
-    for (int t = warp; t < n; t += 4) {
-      const int e = ec + t;
-      const int j = ldg(p.senders + e);
-      if ((unsigned)j >= (unsigned)p.N) {
-        raise_error(p.err, kErrIndex);
-        continue;
-      }
-      T x[D1], y[D2], ph[KP];
-      const T* xr = p.x + (size_t)j * p.c_in + pd.x_off + cl;
+  const int nc = min(kEdgeTile, pd.mul_in - c0), ss = edge_slot_stride(D1 * nc);
+  const int uw = (nc + kEdgeWarps - 1) / kEdgeWarps;
+  const int u0 = warp * uw, u1 = min(nc, u0 + uw);
+  if (u0 >= u1) return;
+  T y[D2], cy[NP], gy[D2];
 #pragma unroll
-      for (int m = 0; m < D1; ++m) x[m] = act ? ldg(xr + (size_t)m * mi) : T(0);
+  for (int m = 0; m < D2; ++m) {
+    y[m] = ok ? ldg(p.Y + (size_t)e * p.dim_y + Y0 + m) : T(0);
+    gy[m] = T(0);
+  }
+  static_for<NP>([&](auto P) { cy[decltype(P)::value] = pair_coef<T, CGp, decltype(P)::value>(y); });
+  const T* xs = Xs + lane * ss;
+  const int srow = nc * p.K;
+  T* ct = CT + lane;   // this lane's column: C[mo], then T_bar[mo]
+#pragma unroll 1
+  for (int u = u0; u < u1; ++u) {
+    T xv[D1];
 #pragma unroll
-      for (int m = 0; m < D2; ++m) y[m] = ldg(p.Y + (size_t)e * p.dim_y + L2 * L2 + m);
-#pragma unroll
-      for (int q = 0; q < KP; ++q) ph[q] = q < p.K ? ldg(p.phi + (size_t)e * p.K + q) : T(0);
+    for (int m = 0; m < D1; ++m) xv[m] = xs[m * nc + u];
+    {
       T C[D3];
 #pragma unroll
       for (int m = 0; m < D3; ++m) C[m] = T(0);
-      static_for<CGp::npair>([&](auto P) {
+      static_for<NP>([&](auto P) {
         constexpr Pair pr = CGp::pair[decltype(P)::value];
-        const T cy = pair_coef<T, CGp, decltype(P)::value>(y);
-        C[pr.m3] = fma(cy, x[pr.m1], C[pr.m3]);
+        C[pr.m3] = fma(cy[decltype(P)::value], xv[pr.m1], C[pr.m3]);
       });
-      T tb[D3], gp[KP];
 #pragma unroll
-      for (int m = 0; m < D3; ++m) tb[m] = T(0);
-#pragma unroll
-      for (int q = 0; q < KP; ++q) {
-        T s = T(0);
-#pragma unroll
-        for (int m = 0; m < D3; ++m) {
-          const T sb = Sb[(q * D3 + m) * 32 + lane];
-          tb[m] = fma(ph[q], sb, tb[m]);
-          s = fma(sb, C[m], s);
-        }
-        gp[q] = s;
-      }
-      T gy[D2];
-#pragma unroll
-      for (int m = 0; m < D2; ++m) gy[m] = T(0);
-      static_for<CGp::npair>([&](auto P) {
-        constexpr Pair pr = CGp::pair[decltype(P)::value];
-        const T z = x[pr.m1] * tb[pr.m3];
-        static_for<pr.n>([&](auto k) {
-          constexpr Term tm = CGp::term[pr.start + decltype(k)::value];
-          gy[tm.m2] = fma(T(tm.c), z, gy[tm.m2]);
-        });
-      });
-      T* a = acc + t * accw;
-#pragma unroll
-      for (int q = 0; q < KP; ++q) {
-        if (q < p.K) {
-          const T v = wsum(gp[q]);
-          if (lane == 0) a[q] += v;
-        }
-      }
-#pragma unroll
-      for (int m = 0; m < D2; ++m) {
-        const T v = wsum(gy[m]);
-        if (lane == 0) a[p.K + L2 * L2 + m] += v;
-      }
+      for (int m = 0; m < D3; ++m) ct[m * 32] = C[m];
     }
-    __syncthreads();
+    const T* su = Ss + u * p.K;
+#pragma unroll 1
+    for (int m = 0; m < D3; ++m) {
+      const T cm = ct[m * 32];
+      const T* sr = su + m * srow;
+      T acc = T(0);
+      if (p.vec) {
+#pragma unroll
+        for (int q = 0; q < KP; q += VW) {
+          if constexpr (VW == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(sr + q);
+            acc = fma(ph[q], v.x, acc); gphi[q] = fma(v.x, cm, gphi[q]);
+            acc = fma(ph[q + 1], v.y, acc); gphi[q + 1] = fma(v.y, cm, gphi[q + 1]);
+            acc = fma(ph[q + 2], v.z, acc); gphi[q + 2] = fma(v.z, cm, gphi[q + 2]);
+            acc = fma(ph[q + 3], v.w, acc); gphi[q + 3] = fma(v.w, cm, gphi[q + 3]);
+          } else {
+            const double2 v = *reinterpret_cast<const double2*>(sr + q);
+            acc = fma(ph[q], v.x, acc); gphi[q] = fma(v.x, cm, gphi[q]);
+            acc = fma(ph[q + 1], v.y, acc); gphi[q + 1] = fma(v.y, cm, gphi[q + 1]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < KP; ++q) {
+          const T v = q < p.K ? sr[q] : T(0);
+          acc = fma(ph[q], v, acc);
+          gphi[q] = fma(v, cm, gphi[q]);
+        }
+      }
+      ct[m * 32] = acc;
+    }
+    T tb[D3];
+#pragma unroll
+    for (int m = 0; m < D3; ++m) tb[m] = ct[m * 32];
+    static_for<NP>([&](auto P) {
+      constexpr Pair pr = CGp::pair[decltype(P)::value];
+      const T z = xv[pr.m1] * tb[pr.m3];
+      static_for<pr.n>([&](auto q) {
+        constexpr Term tm = CGp::term[pr.start + decltype(q)::value];
+        gy[tm.m2] = fma(T(tm.c), z, gy[tm.m2]);
+      });
+    });
   }
+#pragma unroll
+  for (int m = 0; m < D2; ++m) gyr[(Y0 + m) * 32] += gy[m];
+}
+
+template <typename T>
+__device__ __forceinline__ EdgeStage edge_next(const UvwEdgeParams<T>& p, EdgeStage st) {
+  st.c0 += kEdgeTile;
+  if (st.c0 >= p.paths[st.pi].mul_in) {
+    st.c0 = 0;
+    ++st.pi;
+  }
+  return st;
 }
 
 template <typename T, int KP>
-__global__ void __launch_bounds__(kThreads) uvw_edge_kernel(const __grid_constant__ UvwEdgeParams<T> p) {
+__global__ void __launch_bounds__(kEdgeThreads, sizeof(T) == 4 ? 3 : 1)
+uvw_edge_kernel(const __grid_constant__ UvwEdgeParams<T> p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  T* Sb = reinterpret_cast<T*>(smem_raw);                 // [KP][D3max][32]
-  T* acc = Sb + KP * (2 * kLmax + 1) * 32;                // [kEdgeChunk][K + dim_y]
+  T* const buf0 = reinterpret_cast<T*>(smem_raw);   // two stage buffers: x part, then S_bar part
+  const int stage_n = p.smem_stage / (int)sizeof(T), xn = (p.smem_stage - p.smem_sbar) / (int)sizeof(T);
+  T* Red = reinterpret_cast<T*>(smem_raw + 2 * p.smem_stage);                        // [warps][dim_y][32]
+  T* CTs = reinterpret_cast<T*>(smem_raw + 2 * p.smem_stage + p.smem_red);           // [warps][2 kLmax + 1][32]
+  int* js = reinterpret_cast<int*>(smem_raw + 2 * p.smem_stage + p.smem_red + p.smem_ct);   // [32]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int r = p.r0 + blockIdx.x;
-  if (r >= p.N) return;
-  int k0 = ldg(p.rowptr + r), k1 = ldg(p.rowptr + r + 1);
+  if (r >= p.N || p.n_blocks == 0) return;
+  const int k0 = ldg(p.rowptr + r), k1 = ldg(p.rowptr + r + 1);
   if (k0 < 0 || k1 < k0 || k1 > p.E) {
-    raise_error(p.err, kErrCsr);
+    if (threadIdx.x == 0) raise_error(p.err, kErrCsr);
     return;
   }
-  const int accw = p.K + p.dim_y;
-  for (int ec = k0; ec < k1; ec += kEdgeChunk) {
-    const int n = min(kEdgeChunk, k1 - ec);
-    for (int t = threadIdx.x; t < n * accw; t += kThreads) acc[t] = T(0);
-    __syncthreads();
-    for (int b = 0; b < p.n_blocks; ++b) {
-      const UvwBlockD& bd = p.blocks[b];
-      dispatch_l(bd.l, [&](auto L3c) {
+  const int n_paths = p.blocks[p.n_blocks - 1].pend;
+  T* CT = CTs + (size_t)warp * (2 * kLmax + 1) * 32;
+  for (int e0 = k0; e0 < k1; e0 += 32) {
+    const int e = e0 + lane;
+    bool ok = e < k1;
+    int j = 0;
+    if (ok) {
+      j = ldg(p.senders + e);
+      if ((unsigned)j >= (unsigned)p.N) {
+        if (warp == 0) atomicOr(p.err, kErrIndex);
+        ok = false;
+        j = 0;
+      }
+    }
+    __syncthreads();   // the previous round is done with js, the buffers and Red
+    if (warp == 0) js[lane] = j;
+    T ph[KP], gphi[KP];
+#pragma unroll
+    for (int q = 0; q < KP; ++q) {
+      ph[q] = (ok && q < p.K) ? ldg(p.phi + (size_t)e * p.K + q) : T(0);
+      gphi[q] = T(0);
+    }
+    T* gyr = Red + (size_t)warp * p.dim_y * 32 + lane;   // this lane's Y_bar column
+    for (int m = 0; m < p.dim_y; ++m) gyr[m * 32] = T(0);
+    __syncthreads();   // js visible
+    EdgeStage st{0, 0};
+    edge_stage_issue(p, st, r, js, buf0, buf0 + xn);
+    cp_async_commit();
+    for (int s = 0; st.pi < n_paths; ++s) {
+      const EdgeStage nx = edge_next(p, st);
+      T* cur = buf0 + (s & 1) * stage_n;
+      T* nxt = buf0 + ((s + 1) & 1) * stage_n;
+      if (nx.pi < n_paths) edge_stage_issue(p, nx, r, js, nxt, nxt + xn);
+      cp_async_commit();
+      cp_async_wait<1>();   // this stage's copies have landed (own thread)
+      __syncthreads();      // ... and every thread's
+      const PathD& pd = p.paths[st.pi];
+      dispatch_l(pd.l3, [&](auto L3c) {
         constexpr int L3 = decltype(L3c)::value;
-        for (int pi = bd.pbeg; pi < bd.pend; ++pi) {
-          const PathD& pd = p.paths[pi];
-          dispatch_l1l2<L3>(pd.l1, pd.l2, [&](auto A1, auto A2) {
-            edge_path<T, KP, decltype(A1)::value, decltype(A2)::value, L3>(p, bd, pd, r, ec, n, Sb, acc);
-          });
-        }
+        dispatch_l1l2<L3>(pd.l1, pd.l2, [&](auto A1, auto A2) {
+          edge_stage_compute<T, decltype(A1)::value, decltype(A2)::value, L3, KP>(
+              p, pd, st.c0, e, ok, cur, cur + xn, CT, ph, gphi, gyr);
+        });
       });
+      __syncthreads();      // buffer cur is free for the stage after next
+      st = nx;
     }
-    for (int t = threadIdx.x; t < n * accw; t += kThreads) {
-      const int el = t / accw, v = t - el * accw;
-      const int e = ec + el;
-      if (v < p.K)
-        p.gphi[(size_t)e * p.K + v] = acc[t];
-      else
-        p.gY[(size_t)e * p.dim_y + (v - p.K)] = acc[t];
-    }
+    cp_async_wait<0>();
+    // ---- add the warps' partial sums in a fixed order (phi_bar via buffer 0)
+    T* Rp = buf0;   // [warps][K][32]
+#pragma unroll
+    for (int q = 0; q < KP; ++q)
+      if (q < p.K) Rp[((size_t)warp * p.K + q) * 32 + lane] = gphi[q];
     __syncthreads();
+    const int n = min(32, k1 - e0), nv = p.K + p.dim_y;
+    for (int t = threadIdx.x; t < nv * 32; t += kEdgeThreads) {
+      const int v = t >> 5, sl = t & 31;
+      if (sl >= n) continue;
+      const size_t eo = (size_t)e0 + sl;
+      if (v < p.K) {
+        T acc = Rp[(size_t)v * 32 + sl];
+#pragma unroll
+        for (int w = 1; w < kEdgeWarps; ++w) acc += Rp[((size_t)w * p.K + v) * 32 + sl];
+        p.gphi[eo * p.K + v] = acc;
+      } else {
+        const int m = v - p.K;
+        T acc = Red[(size_t)m * 32 + sl];
+#pragma unroll
+        for (int w = 1; w < kEdgeWarps; ++w) acc += Red[((size_t)w * p.dim_y + m) * 32 + sl];
+        p.gY[eo * p.dim_y + m] = acc;
+      }
+    }
   }
 }
 
@@ -312,7 +443,10 @@ __global__ void pack_a_kernel(const __grid_constant__ UvwPackParams p, const T* 
   const PackPath& pp = p.paths[lo];
   const int rem = col - pp.w_off, u = rem / pp.mo, w = rem - u * pp.mo;
   const T v = A[idx];
-  if (Bf) Bf[pp.bf_off + ((size_t)pp.colf + (size_t)q * pp.mi + u) * pp.mo + w] = v;
+  if (Bf) {
+    const size_t rowf = p.bf_uq ? (size_t)u * p.K + q : (size_t)q * pp.mi + u;
+    Bf[pp.bf_off + ((size_t)pp.colf + rowf) * pp.mo + w] = v;
+  }
   if (Ba) Ba[pp.ba_off + ((size_t)pp.cola + (size_t)q * pp.mo + w) * pp.mi + u] = v;
   const T vh = hi_part(v);
   if (Btf) {
@@ -361,11 +495,11 @@ cudaError_t launch_uvw_sbuild_dir(const UvwSParams<T>& p, cudaStream_t s) {
 template <typename T, int KP>
 cudaError_t launch_uvw_edge(const UvwEdgeParams<T>& p, cudaStream_t s) {
   if (p.nr <= 0) return cudaSuccess;
-  const size_t smem = sizeof(T) * ((size_t)KP * (2 * kLmax + 1) * 32 + (size_t)kEdgeChunk * (p.K + p.dim_y));
+  const size_t smem = 2 * (size_t)p.smem_stage + p.smem_red + p.smem_ct + 32 * sizeof(int);
   auto k = uvw_edge_kernel<T, KP>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<p.nr, kThreads, smem, s>>>(p);
+  k<<<p.nr, kEdgeThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
