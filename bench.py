@@ -184,17 +184,42 @@ def roofline_fb(d, ms: float) -> dict:
     return r
 
 
+# DRAM bytes (read + write) per launch of the kernel that a (workload, pass)
+# timing is dominated by, from one ncu capture of the current kernel (the
+# summary under profiles/ names the command); None where no capture of the
+# current kernel exists.
+NCU_TRAFFIC = {
+    (2, 0): (21_649_408 + 680_448, "uvu_fwd_kernel", "profiles/uvu_fwd_kernel_mace_4096.md"),
+}
+
+
 def roofline(d, pass_: int, ms: float) -> dict:
     flops, nbytes = d["plan"].work_model(d["N"], d["E"], pass_)
     dt = d["cfg"].dtype
     peak = alu_peak(dt)
     ach = flops / (ms * 1e-3) / 1e12
-    return {"bound": "alu", "achieved": round(ach, 3), "peak": round(peak, 2), "unit": "TFLOP/s",
-            "frac": round(ach / peak, 4), "traffic": None,
-            "peak_source": f"derived: {SMS} SMs x {FP32_LANES if dt == 'f32' else FP64_LANES} "
-                           f"{'FP32' if dt == 'f32' else 'FP64'} FMA lanes x 2 x {MAX_MHZ:.0f} MHz",
-            "algorithmic_flops": flops, "compulsory_bytes": nbytes,
-            "hbm_frac_of_measured": None}
+    r = {"bound": "alu", "achieved": round(ach, 3), "peak": round(peak, 2), "unit": "TFLOP/s",
+         "frac": round(ach / peak, 4), "traffic": None,
+         "peak_source": f"derived: {SMS} SMs x {FP32_LANES if dt == 'f32' else FP64_LANES} "
+                        f"{'FP32' if dt == 'f32' else 'FP64'} FMA lanes x 2 x {MAX_MHZ:.0f} MHz",
+         "algorithmic_flops": flops, "compulsory_bytes": nbytes,
+         "hbm_frac_of_measured": None}
+    t = NCU_TRAFFIC.get((d["cfg"].id, pass_))
+    if t is not None:
+        hbm = measured_hbm_gbs()
+        r["traffic"] = t[0]
+        r["traffic_source"] = f"{t[1]}: dram__bytes_read.sum + dram__bytes_write.sum, {t[2]}"
+        if hbm:
+            r["hbm_frac_of_measured"] = round(t[0] / (ms * 1e-3) / 1e9 / hbm, 4)
+    return r
+
+
+def measured_hbm_gbs():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"])
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 # ----------------------------------------------------------------------------- CPU oracle

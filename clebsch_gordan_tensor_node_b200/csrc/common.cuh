@@ -82,6 +82,7 @@ struct UvuSrcParams {         // backward: source-owned grad_x, grad_A partials
   int cy_stride;              // cY slots per staged edge (max over tiles, padded)
   int chunk;                  // edges staged per warp at a time (<= 32)
   int warp_smem;              // bytes of shared memory per warp
+  int ring_off, ring_g;       // m_bar copy ring: byte offset in the warp's slice, edges per group
   TileD tiles[kMaxTiles];     // one per (input block, channel tile)
   PathD paths[kMaxPaths];     // grouped by input block
 };

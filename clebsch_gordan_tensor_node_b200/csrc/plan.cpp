@@ -264,9 +264,24 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
     }
     P.src_cy_stride = std::max(P.src_cy_stride, off);
   }
-  P.src_chunk = std::max(1, std::min(32, (20 * 1024) / (P.src_cy_stride * bsz)));
-  P.src_warp_smem = 32 * 4 + 32 * P.KP * bsz + P.src_chunk * P.src_cy_stride * bsz;
-  P.src_warp_smem = (P.src_warp_smem + 15) / 16 * 16;
+  // source pass: per warp, the staged chunk (receivers, radial rows, cY) and an
+  // m_bar copy ring of two groups of ring_g edges (every component of the
+  // widest output block, 32 lanes x CPL channels). Group size, then chunk,
+  // shrink until one CTA of src_warps warps fits on an SM.
+  {
+    const int d3 = 2 * lout + 1, warps = src_warps_for(bsz), budget = 226 * 1024;
+    auto base = [&](int chunk) { return (32 * 4 + 32 * P.KP * bsz + chunk * P.src_cy_stride * bsz + 15) / 16 * 16; };
+    auto per_warp = [&](int chunk, int g) { return base(chunk) + (2 * g * d3 * 32 * P.CPL * bsz + 15) / 16 * 16; };
+    int chunk = std::max(1, std::min(32, (20 * 1024) / (P.src_cy_stride * bsz))), g = 4;
+    while (per_warp(chunk, g) * warps > budget && g > 2) g /= 2;
+    while (per_warp(chunk, g) * warps > budget && chunk > 8) chunk /= 2;
+    while (per_warp(chunk, g) * warps > budget && g > 1) g /= 2;
+    while (per_warp(chunk, g) * warps > budget && chunk > 1) chunk /= 2;
+    P.src_chunk = chunk;
+    P.src_ring_g = g;
+    P.src_ring_off = base(chunk);
+    P.src_warp_smem = per_warp(chunk, g);
+  }
   if (mode == TP_UVW) {
     if ((int)P.bout.size() > kMaxBlocks || (int)P.bin.size() > kMaxBlocks) {
       msg = "more than " + std::to_string(kMaxBlocks) + " irrep blocks";
@@ -368,9 +383,10 @@ int uvw_chunk_rows(const Plan& p, long long n_nodes, int dir) {
 }
 
 int uvu_src_slots(const Plan& p, long long n_nodes) {
-  const long long target = 148LL * 24;  // resident warps to aim for on 148 SMs
+  // one wave of one-CTA-per-SM blocks, each serving one input-block tile
   const long long t = std::max<long long>(1, (long long)p.in_tiles.size());
-  long long s = (target + t - 1) / t;
+  const int w = src_warps_for(p.dtype == TP_F32 ? 4 : 8);
+  long long s = (long long)w * std::max<long long>(1, kSMs / t);
   s = std::min<long long>(s, std::max<long long>(1, n_nodes));
   return (int)s;
 }

@@ -215,7 +215,7 @@ uvu_edge_kernel(const __grid_constant__ UvuEdgeParams<T> p) {
 // block b, channel tile); per chunk of up to 32 outgoing edges, lanes first
 // stage each edge's receiver, radial row and the cY values of every path of b
 // in shared memory; then every path sweeps the chunk with A in registers and
-// the next receiver's m_bar gather in flight. x_bar_j accumulates in registers
+// the receivers' m_bar rows arriving through an asynchronous copy ring. x_bar_j accumulates in registers
 // in one fixed order; the same sweep forms h = <x_j, t'> and adds phi h to the
 // warp's slot of the A_bar partial buffer after each path.
 
@@ -224,7 +224,21 @@ struct SrcSmem {
   int* i;
   T* phi;
   T* cy;
+  T* ring;   // [2][ring_g][2 lmax_out + 1][32 CPL] m_bar rows in flight
 };
+
+// Asynchronous copy of B bytes (4, 8 or 16) from global to shared memory.
+template <int B>
+__device__ __forceinline__ void cp_async_b(void* dst, const void* src) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+  if constexpr (B == 16)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;\n" ::"r"(d), "l"(src), "n"(B) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
 template <typename T, int L1, int L2, int L3>
 __device__ __forceinline__ void src_stage_cy(const T* yrow, T* dst) {
@@ -253,7 +267,6 @@ __device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& 
   using CGp = cgt::CG<L1, L2, L3>;
   constexpr int D1 = 2 * L1 + 1, D3 = 2 * L3 + 1, NP = CGp::npair;
   constexpr int VW = sizeof(T) == 4 ? 4 : 2;
-  constexpr bool kPrefetch = D3 * CPL * sizeof(T) <= 48;
   T a[KP][CPL], ab[KP][CPL];
 #pragma unroll
   for (int q = 0; q < KP; ++q) {
@@ -266,26 +279,42 @@ __device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& 
       for (int c = 0; c < CPL; ++c) a[q][c] = T(0);
     }
   }
+  // m_bar rows of the chunk's receivers go through a two-buffer ring of groups
+  // of ring_g edges: the copies of group g + 1 are in flight while group g is
+  // contracted. Each lane copies and later reads only its own channels.
   const T* gb = p.gout + pd.out_off + chl;
-  const int mo = pd.mul_out;
-  T gv[D3][CPL];
-  if (kPrefetch && n > 0) {
-    const T* gr = gb + (size_t)s.i[0] * p.c_out;
+  const int mo = pd.mul_out, G = p.ring_g, lane = threadIdx.x & 31;
+  constexpr int RW = 32 * CPL;   // ring row: one component of one edge
+  auto issue = [&](int g0, int buf) {
+    for (int t = 0; t < G && g0 + t < n; ++t) {
+      const T* gr = gb + (size_t)s.i[g0 + t] * p.c_out;
+      T* dst = s.ring + ((size_t)(buf * G + t) * D3) * RW + lane * CPL;
 #pragma unroll
-    for (int m = 0; m < D3; ++m) load_ch<CPL>(gv[m], gr + m * mo);
-  }
+      for (int m = 0; m < D3; ++m) cp_async_b<CPL * sizeof(T)>(dst + m * RW, gr + m * mo);
+    }
+  };
+  if (n > 0) issue(0, 0);
+  cp_commit();
   for (int k = 0; k < n; ++k) {
-    T gn[kPrefetch ? D3 : 1][CPL];
-    if constexpr (kPrefetch) {
-      if (k + 1 < n) {
-        const T* gr = gb + (size_t)s.i[k + 1] * p.c_out;
+    const int t = k % G, buf = (k / G) & 1;
+    if (t == 0) {
+      if (k + G < n) issue(k + G, buf ^ 1);
+      cp_commit();
+      cp_wait<1>();   // this group's rows have landed
+    }
+    T gv[D3][CPL];
+    {
+      const T* src = s.ring + ((size_t)(buf * G + t) * D3) * RW + lane * CPL;
 #pragma unroll
-        for (int m = 0; m < D3; ++m) load_ch<CPL>(gn[m], gr + m * mo);
+      for (int m = 0; m < D3; ++m) {
+        if constexpr (CPL == 2 && sizeof(T) == 4) {
+          const float2 v2 = *reinterpret_cast<const float2*>(src + m * RW);
+          gv[m][0] = v2.x; gv[m][1] = v2.y;
+        } else {
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) gv[m][c] = src[m * RW + c];
+        }
       }
-    } else {
-      const T* gr = gb + (size_t)s.i[k] * p.c_out;
-#pragma unroll
-      for (int m = 0; m < D3; ++m) load_ch<CPL>(gv[m], gr + m * mo);
     }
     T ph[KP];
 #pragma unroll
@@ -330,15 +359,8 @@ __device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& 
     for (int q = 0; q < KP; ++q)
 #pragma unroll
       for (int c = 0; c < CPL; ++c) ab[q][c] = fma(ph[q], h[c], ab[q][c]);
-    if constexpr (kPrefetch) {
-      if (k + 1 < n) {
-#pragma unroll
-        for (int m = 0; m < D3; ++m)
-#pragma unroll
-          for (int c = 0; c < CPL; ++c) gv[m][c] = gn[m][c];
-      }
-    }
   }
+  cp_wait<0>();
   if (active && n > 0) {
 #pragma unroll
     for (int q = 0; q < KP; ++q) {
@@ -419,19 +441,24 @@ __device__ __forceinline__ void src_tile(const UvuSrcParams<T>& p, const TileD& 
 }
 
 template <typename T, int KP, int CPL, class PR>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+__global__ void __launch_bounds__(src_warps<T>() * 32, 1)
 uvu_src_kernel(const __grid_constant__ UvuSrcParams<T> p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
+  // every warp of a CTA serves the same input-block tile (one family of path
+  // bodies per SM in the instruction cache); CTAs are tile-major
+  constexpr int W = src_warps<T>();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int wid = blockIdx.x * kWarpsPerBlock + warp;
-  if (wid >= p.n_slots * p.n_tiles) return;
-  const int slot = wid / p.n_tiles;
-  const TileD& tl = p.tiles[wid % p.n_tiles];
+  const int per_tile = (p.n_slots + W - 1) / W;
+  const int tile = blockIdx.x / per_tile;
+  const int slot = (blockIdx.x - tile * per_tile) * W + warp;
+  if (tile >= p.n_tiles || slot >= p.n_slots) return;
+  const TileD& tl = p.tiles[tile];
   unsigned char* base = smem_raw + (size_t)warp * p.warp_smem;
   SrcSmem<T> s;
   s.i = reinterpret_cast<int*>(base);
   s.phi = reinterpret_cast<T*>(base + 32 * sizeof(int));
   s.cy = s.phi + 32 * KP;
+  s.ring = reinterpret_cast<T*>(base + p.ring_off);
   dispatch_l<PR::l1>(tl.l, [&](auto L) { src_tile<T, KP, CPL, PR, decltype(L)::value>(p, tl, slot, lane, s); });
 }
 
@@ -477,13 +504,13 @@ cudaError_t launch_uvu_edge(const UvuEdgeParams<T>& p0, int prof, cudaStream_t s
 
 template <typename T, int KP, int CPL, class PR>
 cudaError_t launch_src_prof(const UvuSrcParams<T>& p, unsigned blocks, cudaStream_t s) {
-  const size_t smem = (size_t)p.warp_smem * kWarpsPerBlock;
+  const size_t smem = (size_t)p.warp_smem * src_warps<T>();
   auto kern = uvu_src_kernel<T, KP, CPL, PR>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  kern<<<blocks, kWarpsPerBlock * 32, smem, s>>>(p);
+  kern<<<blocks, src_warps<T>() * 32, smem, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -491,9 +518,9 @@ template <typename T, int KP, int CPL>
 cudaError_t launch_uvu_src(const UvuSrcParams<T>& p, int prof, cudaStream_t s) {
   cudaError_t err = cudaMemsetAsync(p.apart, 0, sizeof(T) * (size_t)p.n_slots * p.K * p.n_w, s);
   if (err != cudaSuccess) return err;
-  const long long warps = (long long)p.n_slots * p.n_tiles;
-  if (warps == 0 || p.N == 0) return cudaSuccess;
-  const unsigned blocks = (unsigned)((warps + kWarpsPerBlock - 1) / kWarpsPerBlock);
+  if (p.n_slots == 0 || p.n_tiles == 0 || p.N == 0) return cudaSuccess;
+  constexpr int W = src_warps<T>();
+  const unsigned blocks = (unsigned)(((long long)p.n_slots + W - 1) / W * p.n_tiles);
   switch (prof) {
     case 0: return launch_src_prof<T, KP, CPL, Prof<2, 2, 2>>(p, blocks, s);
     case 1: return launch_src_prof<T, KP, CPL, Prof<1, 3, 3>>(p, blocks, s);
