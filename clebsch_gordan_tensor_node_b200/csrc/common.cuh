@@ -10,6 +10,7 @@
 // Indices are int32; scalars are float or double (the plan's dtype).
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <type_traits>
 #include <utility>
@@ -57,6 +58,7 @@ struct UvuFwdParams {
   int cy_stride;              // cY slots per staged edge (max over tiles, padded)
   int chunk;                  // edges staged per warp at a time (<= 32)
   int warp_smem;              // bytes of shared memory per warp
+  int ring_off, ring_g;       // x copy ring: byte offset in the warp's slice, edges per group
   TileD tiles[kMaxTiles];     // one per (output block, channel tile)
   PathD paths[kMaxPaths];     // grouped by output block
 };
@@ -262,6 +264,20 @@ __device__ __forceinline__ void dispatch_l(int l, F&& f) {
 template <typename T>
 __device__ __forceinline__ T ldg(const T* p) { return __ldg(p); }
 
+// Asynchronous copy of B bytes (4, 8 or 16) from global to shared memory, and
+// its commit / wait (per thread: a thread waits only for its own copies).
+template <int B>
+__device__ __forceinline__ void cp_async_b(void* dst, const void* src) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+  if constexpr (B == 16)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;\n" ::"r"(d), "l"(src), "n"(B) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
 // Load CPL consecutive scalars (8-byte aligned when CPL*sizeof(T) == 8).
 template <int CPL, typename T>
 __device__ __forceinline__ void load_ch(T (&v)[CPL], const T* p) {
@@ -321,5 +337,29 @@ __device__ __forceinline__ void load_phi(T (&ph)[KP], const T* row, int K) {
 __device__ __forceinline__ void raise_error(int* err, int bit) {
   if ((threadIdx.x & 31) == 0) atomicOr(err, bit);
 }
+
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on the
+// current device. The attribute call costs host time comparable to a small
+// kernel, so each launcher keeps one SmemLimit per kernel instantiation and
+// the call is made only when a device first needs more than it was given.
+struct SmemLimit {
+  std::atomic<int> granted[64] = {};
+  cudaError_t ensure(const void* kernel, size_t bytes) {
+    if (bytes <= 48 * 1024) return cudaSuccess;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64)
+      return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (granted[dev].load(std::memory_order_acquire) >= (int)bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) {
+      int cur = granted[dev].load();
+      while (cur < (int)bytes && !granted[dev].compare_exchange_weak(cur, (int)bytes)) {
+      }
+    }
+    return e;
+  }
+};
 
 }  // namespace tpc

@@ -245,9 +245,27 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
     }
     P.cy_stride = std::max(P.cy_stride, off);
   }
-  P.fwd_chunk = std::max(1, std::min(32, (20 * 1024) / (P.cy_stride * bsz)));
-  P.fwd_warp_smem = 32 * 4 + 32 * P.KP * bsz + P.fwd_chunk * P.cy_stride * bsz;
-  P.fwd_warp_smem = (P.fwd_warp_smem + 15) / 16 * 16;
+  // forward: per warp, the staged chunk (senders, radial rows, cY) and an x copy
+  // ring of two groups of ring_g edges (every component of the widest input
+  // block, 32 lanes x CPL channels). Group size, then chunk, shrink until one
+  // CTA of fwd_warps warps fits on an SM.
+  {
+    // the kernel sizes the ring for its degree profile's widest input block
+    const int l1p = profs[P.prof][0], d1 = 2 * l1p + 1, warps = fwd_warps_for(bsz), budget = 226 * 1024;
+    const int g = fwd_ring_g(bsz, P.fwd_CPL, l1p);
+    auto base = [&](int chunk) { return (32 * 4 + 32 * P.KP * bsz + chunk * P.cy_stride * bsz + 15) / 16 * 16; };
+    auto per_warp = [&](int chunk) { return base(chunk) + (2 * g * d1 * 32 * P.fwd_CPL * bsz + 15) / 16 * 16; };
+    int chunk = std::max(1, std::min(32, (20 * 1024) / (P.cy_stride * bsz)));
+    while (per_warp(chunk) * warps > budget && chunk > 1) chunk /= 2;
+    if (per_warp(chunk) * warps > budget) {
+      msg = "forward staging exceeds shared memory";
+      return TP_EUNSUPPORTED;
+    }
+    P.fwd_chunk = chunk;
+    P.fwd_ring_g = g;
+    P.fwd_ring_off = base(chunk);
+    P.fwd_warp_smem = per_warp(chunk);
+  }
   // the same staging for the source pass of the backward (paths by input block)
   P.src_cy_stride = vw;
   for (const TileD& t : P.in_tiles) {
@@ -269,18 +287,21 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
   // widest output block, 32 lanes x CPL channels). Group size, then chunk,
   // shrink until one CTA of src_warps warps fits on an SM.
   {
-    const int d3 = 2 * lout + 1, warps = src_warps_for(bsz), budget = 226 * 1024;
+    // the kernel sizes the ring for its degree profile's widest output block
+    const int l3p = profs[P.prof][2], d3 = 2 * l3p + 1, warps = src_warps_for(bsz), budget = 226 * 1024;
+    const int g = src_ring_g(bsz, P.CPL, l3p);
     auto base = [&](int chunk) { return (32 * 4 + 32 * P.KP * bsz + chunk * P.src_cy_stride * bsz + 15) / 16 * 16; };
-    auto per_warp = [&](int chunk, int g) { return base(chunk) + (2 * g * d3 * 32 * P.CPL * bsz + 15) / 16 * 16; };
-    int chunk = std::max(1, std::min(32, (20 * 1024) / (P.src_cy_stride * bsz))), g = 4;
-    while (per_warp(chunk, g) * warps > budget && g > 2) g /= 2;
-    while (per_warp(chunk, g) * warps > budget && chunk > 8) chunk /= 2;
-    while (per_warp(chunk, g) * warps > budget && g > 1) g /= 2;
-    while (per_warp(chunk, g) * warps > budget && chunk > 1) chunk /= 2;
+    auto per_warp = [&](int chunk) { return base(chunk) + (2 * g * d3 * 32 * P.CPL * bsz + 15) / 16 * 16; };
+    int chunk = std::max(1, std::min(32, (20 * 1024) / (P.src_cy_stride * bsz)));
+    while (per_warp(chunk) * warps > budget && chunk > 1) chunk /= 2;
+    if (per_warp(chunk) * warps > budget) {
+      msg = "source-pass staging exceeds shared memory";
+      return TP_EUNSUPPORTED;
+    }
     P.src_chunk = chunk;
     P.src_ring_g = g;
     P.src_ring_off = base(chunk);
-    P.src_warp_smem = per_warp(chunk, g);
+    P.src_warp_smem = per_warp(chunk);
   }
   if (mode == TP_UVW) {
     if ((int)P.bout.size() > kMaxBlocks || (int)P.bin.size() > kMaxBlocks) {

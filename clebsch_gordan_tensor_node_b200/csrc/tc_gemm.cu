@@ -325,8 +325,8 @@ size_t tc_smem_bytes(int npmax) {
 cudaError_t launch_gemm_tc(const TcBatch& tb, int n_prob, int max_m, int npmax, int* err, cudaStream_t s) {
   if (n_prob == 0 || max_m == 0) return cudaSuccess;
   const size_t smem = tc_smem_bytes(npmax);
-  cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  static SmemLimit limit;
+  if (cudaError_t e = limit.ensure((const void*)tc_gemm_kernel, smem); e != cudaSuccess) return e;
   dim3 grid((max_m + TM - 1) / TM, n_prob);
   tc_gemm_kernel<<<grid, 128, smem, s>>>(tb, npmax, err);
   return cudaGetLastError();

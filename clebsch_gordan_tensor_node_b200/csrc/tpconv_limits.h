@@ -21,4 +21,30 @@ __host__ __device__
 #endif
 constexpr int src_warps() { return src_warps_for(sizeof(T)); }
 
+// Warps per CTA of the uvu forward, also one CTA per SM.
+#ifdef __CUDACC__
+__host__ __device__
+#endif
+constexpr int fwd_warps_for(int scalar_bytes) { return scalar_bytes == 4 ? 16 : 8; }
+template <typename T>
+#ifdef __CUDACC__
+__host__ __device__
+#endif
+constexpr int fwd_warps() { return fwd_warps_for(sizeof(T)); }
+
+// Edges per group of the forward's x copy ring (two groups per warp in
+// flight): 4 while the widest input block has at most 3 components, else 2,
+// which leaves shared memory for a full 32-edge staged chunk (the ring restarts
+// with every path of every chunk, so long chunks matter more than deep groups).
+#ifdef __CUDACC__
+__host__ __device__
+#endif
+constexpr int fwd_ring_g(int scalar_bytes, int cpl, int l1max) { return l1max <= 1 ? 4 : 2; }
+
+// The same for the source pass's m_bar ring (widest output block, degree l3max).
+#ifdef __CUDACC__
+__host__ __device__
+#endif
+constexpr int src_ring_g(int scalar_bytes, int cpl, int l3max) { return l3max <= 1 ? 4 : 2; }
+
 }  // namespace tpc

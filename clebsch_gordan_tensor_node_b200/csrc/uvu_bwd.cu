@@ -224,21 +224,9 @@ struct SrcSmem {
   int* i;
   T* phi;
   T* cy;
-  T* ring;   // [2][ring_g][2 lmax_out + 1][32 CPL] m_bar rows in flight
+  T* ring;   // [2][G][2 lmax_out + 1][32 CPL] m_bar rows in flight
 };
 
-// Asynchronous copy of B bytes (4, 8 or 16) from global to shared memory.
-template <int B>
-__device__ __forceinline__ void cp_async_b(void* dst, const void* src) {
-  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
-  if constexpr (B == 16)
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src) : "memory");
-  else
-    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;\n" ::"r"(d), "l"(src), "n"(B) : "memory");
-}
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
 template <typename T, int L1, int L2, int L3>
 __device__ __forceinline__ void src_stage_cy(const T* yrow, T* dst) {
@@ -260,7 +248,7 @@ __device__ __forceinline__ void lds16(T* v, const T* src) {
   }
 }
 
-template <typename T, int KP, int CPL, int L1, int L2, int L3>
+template <typename T, int KP, int CPL, int G, int L1, int L2, int L3>
 __device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& pd, const SrcSmem<T>& s, int n,
                                          int slot, int chl, bool active, const T (&xs)[2 * L1 + 1][CPL],
                                          T (&gx)[2 * L1 + 1][CPL]) {
@@ -283,28 +271,32 @@ __device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& 
   // of ring_g edges: the copies of group g + 1 are in flight while group g is
   // contracted. Each lane copies and later reads only its own channels.
   const T* gb = p.gout + pd.out_off + chl;
-  const int mo = pd.mul_out, G = p.ring_g, lane = threadIdx.x & 31;
+  const int mo = pd.mul_out, lane = threadIdx.x & 31;
   constexpr int RW = 32 * CPL;   // ring row: one component of one edge
   auto issue = [&](int g0, int buf) {
-    for (int t = 0; t < G && g0 + t < n; ++t) {
-      const T* gr = gb + (size_t)s.i[g0 + t] * p.c_out;
-      T* dst = s.ring + ((size_t)(buf * G + t) * D3) * RW + lane * CPL;
 #pragma unroll
-      for (int m = 0; m < D3; ++m) cp_async_b<CPL * sizeof(T)>(dst + m * RW, gr + m * mo);
+    for (int t = 0; t < G; ++t) {
+      if (g0 + t < n) {
+        const T* gr = gb + (size_t)s.i[g0 + t] * p.c_out;
+        T* dst = s.ring + ((buf * G + t) * D3) * RW + lane * CPL;
+#pragma unroll
+        for (int m = 0; m < D3; ++m) cp_async_b<CPL * sizeof(T)>(dst + m * RW, gr + m * mo);
+      }
     }
   };
   if (n > 0) issue(0, 0);
   cp_commit();
-  for (int k = 0; k < n; ++k) {
-    const int t = k % G, buf = (k / G) & 1;
-    if (t == 0) {
-      if (k + G < n) issue(k + G, buf ^ 1);
-      cp_commit();
-      cp_wait<1>();   // this group's rows have landed
-    }
+  for (int g0 = 0, buf = 0; g0 < n; g0 += G, buf ^= 1) {
+    if (g0 + G < n) issue(g0 + G, buf ^ 1);
+    cp_commit();
+    cp_wait<1>();   // this group's rows have landed
+    const int tn = min(G, n - g0);
+#pragma unroll 1
+  for (int t = 0; t < tn; ++t) {
+    const int k = g0 + t;
     T gv[D3][CPL];
     {
-      const T* src = s.ring + ((size_t)(buf * G + t) * D3) * RW + lane * CPL;
+      const T* src = s.ring + ((buf * G + t) * D3) * RW + lane * CPL;
 #pragma unroll
       for (int m = 0; m < D3; ++m) {
         if constexpr (CPL == 2 && sizeof(T) == 4) {
@@ -359,6 +351,7 @@ __device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& 
     for (int q = 0; q < KP; ++q)
 #pragma unroll
       for (int c = 0; c < CPL; ++c) ab[q][c] = fma(ph[q], h[c], ab[q][c]);
+  }
   }
   cp_wait<0>();
   if (active && n > 0) {
@@ -426,8 +419,8 @@ __device__ __forceinline__ void src_tile(const UvuSrcParams<T>& p, const TileD& 
         const PathD& pd = p.paths[pi];
         dispatch_l2l3<L1, PR::l2>(pd.l2, pd.l3, [&](auto A2, auto A3) {
           if constexpr (decltype(A3)::value <= PR::l3)
-            src_path<T, KP, CPL, L1, decltype(A2)::value, decltype(A3)::value>(p, pd, s, n, slot, chl, active, xs,
-                                                                               gx);
+            src_path<T, KP, CPL, src_ring_g(sizeof(T), CPL, PR::l3), L1, decltype(A2)::value,
+                     decltype(A3)::value>(p, pd, s, n, slot, chl, active, xs, gx);
         });
       }
       __syncwarp();
@@ -477,10 +470,8 @@ __global__ void reduce_slots_kernel(const T* __restrict__ part, T* __restrict__ 
 template <typename T, int KP, int V, class PR>
 cudaError_t launch_edge_prof(const UvuEdgeParams<T>& p, unsigned blocks, size_t smem, cudaStream_t s) {
   auto kern = uvu_edge_kernel<T, KP, V, PR>;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
+  static SmemLimit limit;
+  if (cudaError_t e = limit.ensure((const void*)kern, smem); e != cudaSuccess) return e;
   kern<<<blocks, kWarpsPerBlock * 32, smem, s>>>(p);
   return cudaGetLastError();
 }
@@ -506,10 +497,8 @@ template <typename T, int KP, int CPL, class PR>
 cudaError_t launch_src_prof(const UvuSrcParams<T>& p, unsigned blocks, cudaStream_t s) {
   const size_t smem = (size_t)p.warp_smem * src_warps<T>();
   auto kern = uvu_src_kernel<T, KP, CPL, PR>;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
+  static SmemLimit limit;
+  if (cudaError_t e = limit.ensure((const void*)kern, smem); e != cudaSuccess) return e;
   kern<<<blocks, src_warps<T>() * 32, smem, s>>>(p);
   return cudaGetLastError();
 }

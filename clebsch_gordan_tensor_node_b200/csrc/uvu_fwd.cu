@@ -19,8 +19,8 @@
 // Edges are processed in chunks of up to 32: first each lane takes one edge of
 // the chunk and writes its sender, radial row and the cY values of every path
 // of the tile into the warp's shared-memory slice; then the warp sweeps the
-// chunk once per path, reading those values as broadcasts while the gather of
-// the next sender's x row is already in flight.
+// chunk once per path, reading those values as broadcasts while the x rows of
+// the next group of senders arrive through an asynchronous copy ring.
 //
 // Task order: windows of kWin receivers; inside a window all receivers of one
 // tile come first, so the warps of a CTA run the same code on neighbouring
@@ -38,6 +38,7 @@ struct FwdSmem {
   int* j;
   T* phi;
   T* cy;
+  T* ring;   // [2][ring_g][2 lmax_in + 1][32 CPL] x rows in flight
 };
 
 template <typename T, int KP>
@@ -48,6 +49,7 @@ __device__ __forceinline__ FwdSmem<T> fwd_smem(const UvuFwdParams<T>& p, int war
   s.j = reinterpret_cast<int*>(base);
   s.phi = reinterpret_cast<T*>(base + 32 * sizeof(int));
   s.cy = s.phi + 32 * KP;
+  s.ring = reinterpret_cast<T*>(base + p.ring_off);
   return s;
 }
 
@@ -73,14 +75,12 @@ __device__ __forceinline__ void lds16(T* v, const T* src) {
   }
 }
 
-template <typename T, int KP, int CPL, int L1, int L2, int L3>
+template <typename T, int KP, int CPL, int G, int L1, int L2, int L3>
 __device__ __forceinline__ void fwd_path(const UvuFwdParams<T>& p, const PathD& pd, const FwdSmem<T>& s,
                                          int n, int chl, T (&acc)[2 * L3 + 1][CPL]) {
   using CGp = cgt::CG<L1, L2, L3>;
   constexpr int D1 = 2 * L1 + 1, D3 = 2 * L3 + 1, NP = CGp::npair;
   constexpr int VW = sizeof(T) == 4 ? 4 : 2;           // scalars per 16-byte shared load
-  // double-buffer the x gather only while the buffer stays small
-  constexpr bool kPrefetch = D1 * CPL * sizeof(T) <= 48;
   T a[KP][CPL];
 #pragma unroll
   for (int q = 0; q < KP; ++q) {
@@ -91,27 +91,46 @@ __device__ __forceinline__ void fwd_path(const UvuFwdParams<T>& p, const PathD& 
       for (int c = 0; c < CPL; ++c) a[q][c] = T(0);
     }
   }
+  // x rows of the chunk's senders go through a two-buffer ring of groups of G
+  // edges: the copies of group g + 1 are in flight while group g is
+  // contracted. Each lane copies and later reads only its own channels.
   const T* xb = p.x + pd.x_off + chl;
-  const int mul = pd.mul_in;
-  T xv[D1][CPL];
-  if (kPrefetch && n > 0) {
-    const T* xr = xb + (size_t)s.j[0] * p.c_in;
+  const int mul = pd.mul_in, lane = threadIdx.x & 31;
+  constexpr int RW = 32 * CPL;   // ring row: one component of one edge
+  auto issue = [&](int g0, int buf) {
 #pragma unroll
-    for (int m = 0; m < D1; ++m) load_ch<CPL>(xv[m], xr + m * mul);
-  }
-  for (int k = 0; k < n; ++k) {
-    T xn[kPrefetch ? D1 : 1][CPL];
-    if constexpr (kPrefetch) {
-      // gather of the next edge's x row, in flight during this edge's arithmetic
-      if (k + 1 < n) {
-        const T* xr = xb + (size_t)s.j[k + 1] * p.c_in;
+    for (int t = 0; t < G; ++t) {
+      if (g0 + t < n) {
+        const T* xr = xb + (size_t)s.j[g0 + t] * p.c_in;
+        T* dst = s.ring + ((buf * G + t) * D1) * RW + lane * CPL;
 #pragma unroll
-        for (int m = 0; m < D1; ++m) load_ch<CPL>(xn[m], xr + m * mul);
+        for (int m = 0; m < D1; ++m) cp_async_b<CPL * sizeof(T)>(dst + m * RW, xr + m * mul);
       }
-    } else {
-      const T* xr = xb + (size_t)s.j[k] * p.c_in;
+    }
+  };
+  if (n > 0) issue(0, 0);
+  cp_commit();
+  for (int g0 = 0, buf = 0; g0 < n; g0 += G, buf ^= 1) {
+    if (g0 + G < n) issue(g0 + G, buf ^ 1);
+    cp_commit();
+    cp_wait<1>();   // this group's rows have landed
+    const int tn = min(G, n - g0);
+#pragma unroll 1
+  for (int t = 0; t < tn; ++t) {
+    const int k = g0 + t;
+    T xv[D1][CPL];
+    {
+      const T* src = s.ring + ((buf * G + t) * D1) * RW + lane * CPL;
 #pragma unroll
-      for (int m = 0; m < D1; ++m) load_ch<CPL>(xv[m], xr + m * mul);
+      for (int m = 0; m < D1; ++m) {
+        if constexpr (CPL == 2 && sizeof(T) == 4) {
+          const float2 v2 = *reinterpret_cast<const float2*>(src + m * RW);
+          xv[m][0] = v2.x; xv[m][1] = v2.y;
+        } else {
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) xv[m][c] = src[m * RW + c];
+        }
+      }
     }
     T ph[KP];
 #pragma unroll
@@ -161,15 +180,9 @@ __device__ __forceinline__ void fwd_path(const UvuFwdParams<T>& p, const PathD& 
         }
       });
     }
-    if constexpr (kPrefetch) {
-      if (k + 1 < n) {
-#pragma unroll
-        for (int m = 0; m < D1; ++m)
-#pragma unroll
-          for (int c = 0; c < CPL; ++c) xv[m][c] = xn[m][c];
-      }
-    }
   }
+  }
+  cp_wait<0>();
 }
 
 template <typename T, int KP, int CPL, int L1M, int L2M, int L3>
@@ -219,7 +232,8 @@ __device__ __forceinline__ void fwd_tile(const UvuFwdParams<T>& p, const TileD& 
     for (int pi = tl.pbeg; pi < tl.pend; ++pi) {
       const PathD& pd = p.paths[pi];
       dispatch_l1l2<L3, L1M, L2M>(pd.l1, pd.l2, [&](auto A1, auto A2) {
-        fwd_path<T, KP, CPL, decltype(A1)::value, decltype(A2)::value, L3>(p, pd, s, n, chl, acc);
+        fwd_path<T, KP, CPL, fwd_ring_g(sizeof(T), CPL, L1M), decltype(A1)::value, decltype(A2)::value, L3>(
+            p, pd, s, n, chl, acc);
       });
     }
     __syncwarp();
@@ -231,13 +245,13 @@ __device__ __forceinline__ void fwd_tile(const UvuFwdParams<T>& p, const TileD& 
   }
 }
 
-// fp32: two CTAs per SM (register cap 128) measured faster than one CTA with
-// more registers; fp64 spills under that cap, so it keeps one.
+// One CTA per SM: 16 warps (fp32; a 128-register cap) or 8 (fp64), all of one
+// tile's path family at a time.
 template <typename T, int KP, int CPL, int L1M, int L2M, int L3M>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32, sizeof(T) == 4 ? 2 : 1)
+__global__ void __launch_bounds__(fwd_warps<T>() * 32, 1)
 uvu_fwd_kernel(const __grid_constant__ UvuFwdParams<T> p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const long long task = (long long)blockIdx.x * kWarpsPerBlock + warp;
+  const long long task = (long long)blockIdx.x * fwd_warps<T>() + warp;
   const long long per_win = (long long)kWin * p.n_tiles;
   const long long win = task / per_win;
   const int r = (int)(task - win * per_win);
@@ -258,14 +272,13 @@ cudaError_t launch_uvu_fwd(const UvuFwdParams<T>& p, cudaStream_t s) {
   const long long wins = ((long long)p.N + kWin - 1) / kWin;
   const long long tasks = wins * kWin * p.n_tiles;
   if (tasks == 0) return cudaSuccess;
-  const long long blocks = (tasks + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  const size_t smem = (size_t)p.warp_smem * kWarpsPerBlock;
+  constexpr int W = fwd_warps<T>();
+  const long long blocks = (tasks + W - 1) / W;
+  const size_t smem = (size_t)p.warp_smem * W;
   auto kern = uvu_fwd_kernel<T, KP, CPL, L1M, L2M, L3M>;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  kern<<<(unsigned)blocks, kWarpsPerBlock * 32, smem, s>>>(p);
+  static SmemLimit limit;
+  if (cudaError_t e = limit.ensure((const void*)kern, smem); e != cudaSuccess) return e;
+  kern<<<(unsigned)blocks, W * 32, smem, s>>>(p);
   return cudaGetLastError();
 }
 

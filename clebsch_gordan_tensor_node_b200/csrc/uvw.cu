@@ -486,8 +486,8 @@ cudaError_t launch_uvw_sbuild_dir(const UvwSParams<T>& p, cudaStream_t s) {
   const size_t smem = sizeof(T) * (size_t)(kChunk * (2 * kLmax + 1) * 32 + kChunk * KP);
   dim3 grid(p.nr, p.n_blocks);
   auto k = uvw_sbuild_kernel<T, KP, DIR>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  static SmemLimit limit;
+  if (cudaError_t e = limit.ensure((const void*)k, smem); e != cudaSuccess) return e;
   k<<<grid, kThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
@@ -497,8 +497,8 @@ cudaError_t launch_uvw_edge(const UvwEdgeParams<T>& p, cudaStream_t s) {
   if (p.nr <= 0) return cudaSuccess;
   const size_t smem = 2 * (size_t)p.smem_stage + p.smem_red + p.smem_ct + 32 * sizeof(int);
   auto k = uvw_edge_kernel<T, KP>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  static SmemLimit limit;
+  if (cudaError_t e = limit.ensure((const void*)k, smem); e != cudaSuccess) return e;
   k<<<p.nr, kEdgeThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
