@@ -279,6 +279,7 @@ int backward_uvw(const Plan& P, const void* x, const void* Y, const void* phi, c
   const size_t s0 = align256((size_t)NR * P.s_row_elems * b), s1 = align256((size_t)NS * P.sa_row_elems * b);
   T* S = (T*)((char*)ws + na * a);
   T* Sb = (T*)((char*)ws + na * a + std::max(s0, s1));
+  T* Apart = (T*)((char*)ws + na * a + 2 * std::max(s0, s1));   // kTnSplits copies of the A_bar layout
   // Bf feeds only S_bar = m_bar Bf^T here: rows in (u, q) order give S_bar the
   // column order of the edge pass
   UvwPackParams pk = P.pack;
@@ -362,11 +363,16 @@ int backward_uvw(const Plan& P, const void* x, const void* Y, const void* phi, c
           mm = std::max(mm, q.M); mn = std::max(mn, q.D);
         }
         if (n == kMaxGemmBatch || g + 1 == P.uvw_out.size()) {
-          if ((e = launch_gemm<T>(pass == 0 ? 2 : 1, gb, n, mm, mn, s)) != cudaSuccess)
-            return cuda_fail(e, "uvw backward GEMM");
+          e = pass == 0 ? launch_gemm_tn_split<T>(gb, n, mm, mn, Ab, Apart, a / b, kTnSplits, s)
+                        : launch_gemm_nt<T>(gb, n, mm, mn, s);
+          if (e != cudaSuccess) return cuda_fail(e, "uvw backward GEMM");
           n = mm = mn = 0;
         }
       }
+      // A_bar (+)= the split partials, in split order
+      if (pass == 0 && (e = launch_sum_splits<T>(Apart, a / b, kTnSplits, Ab, (long long)P.K * P.n_w, r0 > 0, s)) !=
+                           cudaSuccess)
+        return cuda_fail(e, "uvw A_bar split sum");
     }
     ep.r0 = r0;
     ep.nr = nr;

@@ -39,6 +39,16 @@ cudaError_t launch_unpack_a(const UvwPackParams& p, const T* Bf, T* A, cudaStrea
 // op 0: C = X B (C row-blocked); op 1: C = G B^T (dense); op 2: C (+)= X^T G (dense)
 template <typename T>
 cudaError_t launch_gemm(int op, const GemmBatch<T>& gb, int n_prob, int max_m, int max_n, cudaStream_t s);
+// backward products: S_bar = m_bar B^T, and the split-K A_bar partials with
+// their fixed-order sum (kTnSplits partial copies of the packed-A layout)
+template <typename T>
+cudaError_t launch_gemm_nt(const GemmBatch<T>& gb, int n_prob, int max_m, int max_d, cudaStream_t s);
+template <typename T>
+cudaError_t launch_gemm_tn_split(const GemmBatch<T>& gb, int n_prob, int max_d, int max_n, const T* c_base,
+                                 T* partial, size_t split_stride, int splits, cudaStream_t s);
+template <typename T>
+cudaError_t launch_sum_splits(const T* partial, size_t split_stride, int splits, T* out, long long n, int accumulate,
+                              cudaStream_t s);
 
 // op 0 on tensor cores (fp32, 3xTF32): C = X Bt^T with X [M, D] and Bt [N, D]
 // row-major, read through TMA tensor maps (box 32 x 128 for X, 32 x N16 for Bt).

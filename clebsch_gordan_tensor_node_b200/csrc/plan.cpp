@@ -424,8 +424,9 @@ size_t workspace_bytes(const Plan& p, long long n_nodes, int pass) {
     const size_t a = ((size_t)p.K * p.n_w * b + 255) / 256 * 256;
     const size_t s0 = ((size_t)uvw_chunk_rows(p, n_nodes, 0) * p.s_row_elems * b + 255) / 256 * 256;
     const size_t s1 = ((size_t)uvw_chunk_rows(p, n_nodes, 1) * p.sa_row_elems * b + 255) / 256 * 256;
-    // the tensor-core path adds the low parts of the transposed operands
-    const size_t na = pass == 0 ? (p.uvw_tc ? 2 : 1) : (p.uvw_tc ? 4 : 3);
+    // the tensor-core path adds the low parts of the transposed operands; the
+    // backward adds the split-K partials of A_bar
+    const size_t na = pass == 0 ? (p.uvw_tc ? 2 : 1) : (p.uvw_tc ? 4 : 3) + kTnSplits;
     bytes = na * a + (pass == 0 ? s0 : 2 * std::max(s0, s1));
   }
   return (bytes + 255) / 256 * 256;

@@ -8,6 +8,7 @@ constexpr int kMaxPaths = 192;    // paths per plan (kernel parameter space)
 constexpr int kMaxTiles = 96;     // (block, channel tile) pairs per plan
 constexpr int kWarpsPerBlock = 8; // warps per CTA of the warp-task kernels
 constexpr int kSMs = 148;         // streaming multiprocessors of a B200
+constexpr int kTnSplits = 8;      // split-K partial copies of A_bar in the uvw backward
 
 // Warps per CTA of the uvu source pass, which runs one CTA per SM: 16 for fp32,
 // 8 for fp64 (whose path bodies need more than 128 registers per thread).
