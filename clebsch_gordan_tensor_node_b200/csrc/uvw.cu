@@ -34,8 +34,32 @@ struct SbSmem {
   T* phi;   // [kChunk][KP]
 };
 
+// One m16n8k8 tensor-core product with tf32 operands and fp32 accumulation.
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const unsigned (&a)[4], const unsigned (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// x = hi + lo with hi holding the top 19 bits (a tf32 value) and lo the exact
+// remainder; the tensor core reads lo's top 19 bits.
+__device__ __forceinline__ void split_tf32(float x, unsigned& hi, unsigned& lo) {
+  hi = __float_as_uint(x) & 0xFFFFE000u;
+  lo = __float_as_uint(x - __uint_as_float(hi));
+}
+
 // One path of one owner block: accumulate the state columns (q, channel) of
-// this warp's radial indices over the owner's edges, then store them.
+// this CTA's channel tile over the owner's edges, then store them.
+//
+// Phase A (all types): the warps contract the CG product C[e][mo][u] of the
+// chunk's edges into shared memory, lane = channel u.
+// Phase B, fp32: S[q][(mo, u)] += sum_e phi[e][q] C[e][mo][u] is a product with
+// 16 rows (q), 32 DO columns and the chunk's edges as inner dimension; it runs
+// on the tensor cores as m16n8k8 tf32 products in three parts (hi*hi + hi*lo +
+// lo*hi, the fp32-accurate split), warp w owning channels 8w .. 8w + 7 of every
+// component. fp64: warp w owns radial indices 4w .. 4w + 3, lane = channel,
+// plain FMAs.
 template <typename T, int KP, int DIR, int L1, int L2, int L3>
 __device__ __forceinline__ void sbuild_path(const UvwSParams<T>& p, const UvwBlockD& bd, const PathD& pd,
                                             int r, int k0, int k1, T* Cs, T* phis) {
@@ -44,16 +68,24 @@ __device__ __forceinline__ void sbuild_path(const UvwSParams<T>& p, const UvwBlo
   constexpr int DG = DIR == 0 ? D1 : D3;   // components of the gathered block
   constexpr int DO = DIR == 0 ? D3 : D1;   // components of the owner block
   constexpr int KQ = KP / 4;
+  constexpr bool kTC = sizeof(T) == 4;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;   // mma fragment coordinates
   const int gmul = pd.mul_in;              // gathered multiplicity (direction-specific)
   for (int c0 = 0; c0 < gmul; c0 += 32) {
     const bool act = c0 + lane < gmul;
     const int cl = act ? c0 + lane : c0;
-    T Sr[KQ][DO];
+    T Sr[kTC ? 1 : KQ][DO];                  // fp64 accumulators
+    float acc[kTC ? DO : 1][4];              // fp32: [component][mma C fragment]
 #pragma unroll
-    for (int q = 0; q < KQ; ++q)
+    for (int m = 0; m < DO; ++m) {
+      if constexpr (kTC) {
+        acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.f;
+      } else {
 #pragma unroll
-      for (int m = 0; m < DO; ++m) Sr[q][m] = T(0);
+        for (int q = 0; q < KQ; ++q) Sr[q][m] = T(0);
+      }
+    }
     for (int kc = k0; kc < k1; kc += kChunk) {
       const int n = min(kChunk, k1 - kc);
       // phase A: warp w contracts the CG product of chunk edges w, w+4, ...
@@ -85,29 +117,81 @@ __device__ __forceinline__ void sbuild_path(const UvwSParams<T>& p, const UvwBlo
         for (int m = 0; m < DO; ++m) Cs[(t * DO + m) * 32 + lane] = (act && ok) ? C[m] : T(0);
         if (lane < KP) phis[t * KP + lane] = (ok && lane < p.K) ? ldg(p.phi + (size_t)e * p.K + lane) : T(0);
       }
+      if constexpr (kTC) {
+        // zero rows up to the next multiple of 8 edges (the last mma step)
+        const int n8 = (n + 7) & ~7;
+        for (int t = n + warp; t < n8; t += 4) {
+#pragma unroll
+          for (int m = 0; m < DO; ++m) Cs[(t * DO + m) * 32 + lane] = T(0);
+          if (lane < KP) phis[t * KP + lane] = T(0);
+        }
+      }
       __syncthreads();
-      // phase B: S[q][m] += phi[q] C[m] for this warp's radial indices
-      for (int t = 0; t < n; ++t) {
-        T cm[DO];
+      if constexpr (kTC) {
+        // phase B on the tensor cores: A = phi^T (16 x 8 edges), B = C (8 edges x 8 channels)
+        const float* Cf = reinterpret_cast<const float*>(Cs);
+        const float* Pf = reinterpret_cast<const float*>(phis);
+        for (int e0 = 0; e0 < n; e0 += 8) {
+          unsigned ah[4], al[4];
+          {
+            const int ea = e0 + tig, eb = e0 + tig + 4;
+            const float v0 = gid < KP ? Pf[ea * KP + gid] : 0.f;
+            const float v1 = gid + 8 < KP ? Pf[ea * KP + gid + 8] : 0.f;
+            const float v2 = gid < KP ? Pf[eb * KP + gid] : 0.f;
+            const float v3 = gid + 8 < KP ? Pf[eb * KP + gid + 8] : 0.f;
+            split_tf32(v0, ah[0], al[0]);
+            split_tf32(v1, ah[1], al[1]);
+            split_tf32(v2, ah[2], al[2]);
+            split_tf32(v3, ah[3], al[3]);
+          }
 #pragma unroll
-        for (int m = 0; m < DO; ++m) cm[m] = Cs[(t * DO + m) * 32 + lane];
+          for (int m = 0; m < DO; ++m) {
+            unsigned bh[2], bl[2];
+            split_tf32(Cf[((e0 + tig) * DO + m) * 32 + warp * 8 + gid], bh[0], bl[0]);
+            split_tf32(Cf[((e0 + tig + 4) * DO + m) * 32 + warp * 8 + gid], bh[1], bl[1]);
+            mma_tf32(acc[m], al, bh);
+            mma_tf32(acc[m], ah, bl);
+            mma_tf32(acc[m], ah, bh);
+          }
+        }
+      } else {
+        // phase B: S[q][m] += phi[q] C[m] for this warp's radial indices
+        for (int t = 0; t < n; ++t) {
+          T cm[DO];
 #pragma unroll
-        for (int q = 0; q < KQ; ++q) {
-          const T ph = phis[t * KP + warp * KQ + q];
+          for (int m = 0; m < DO; ++m) cm[m] = Cs[(t * DO + m) * 32 + lane];
 #pragma unroll
-          for (int m = 0; m < DO; ++m) Sr[q][m] = fma(ph, cm[m], Sr[q][m]);
+          for (int q = 0; q < KQ; ++q) {
+            const T ph = phis[t * KP + warp * KQ + q];
+#pragma unroll
+            for (int m = 0; m < DO; ++m) Sr[q][m] = fma(ph, cm[m], Sr[q][m]);
+          }
         }
       }
       __syncthreads();
     }
-    if (act) {
-      T* dst = p.S + (size_t)p.nr_alloc * bd.s_off + (size_t)(r - p.r0) * DO * bd.dcols + pd.col_off + cl;
+    T* dst = p.S + (size_t)p.nr_alloc * bd.s_off + (size_t)(r - p.r0) * DO * bd.dcols + pd.col_off;
+    if constexpr (kTC) {
+      // C fragment: rows q = gid, gid + 8; columns u = 8 warp + 2 tig, + 1
+      const int u = c0 + warp * 8 + 2 * tig;
+#pragma unroll
+      for (int m = 0; m < DO; ++m) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int q = gid + 8 * h;
+          if (q >= p.K) continue;
+          T* row = dst + (size_t)m * bd.dcols + (size_t)q * gmul;
+          if (u < gmul) row[u] = acc[m][2 * h];
+          if (u + 1 < gmul) row[u + 1] = acc[m][2 * h + 1];
+        }
+      }
+    } else if (act) {
 #pragma unroll
       for (int q = 0; q < KQ; ++q) {
         const int qq = warp * KQ + q;
         if (qq < p.K) {
 #pragma unroll
-          for (int m = 0; m < DO; ++m) dst[(size_t)m * bd.dcols + (size_t)qq * gmul] = Sr[q][m];
+          for (int m = 0; m < DO; ++m) dst[(size_t)m * bd.dcols + (size_t)qq * gmul + cl] = Sr[q][m];
         }
       }
     }
