@@ -251,7 +251,8 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
   // CTA of fwd_warps warps fits on an SM.
   {
     // the kernel sizes the ring for its degree profile's widest input block
-    const int l1p = profs[P.prof][0], d1 = 2 * l1p + 1, warps = fwd_warps_for(bsz), budget = 226 * 1024;
+    const int l1p = profs[P.prof][0], d1 = 2 * l1p + 1, warps = fwd_warps_for(bsz);
+    const int budget = 226 * 1024 / ctas_per_sm_for(bsz);
     const int g = fwd_ring_g(bsz, P.fwd_CPL, l1p);
     auto base = [&](int chunk) { return (32 * 4 + 32 * P.KP * bsz + chunk * P.cy_stride * bsz + 15) / 16 * 16; };
     auto per_warp = [&](int chunk) { return base(chunk) + (2 * g * d1 * 32 * P.fwd_CPL * bsz + 15) / 16 * 16; };
@@ -288,7 +289,8 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
   // shrink until one CTA of src_warps warps fits on an SM.
   {
     // the kernel sizes the ring for its degree profile's widest output block
-    const int l3p = profs[P.prof][2], d3 = 2 * l3p + 1, warps = src_warps_for(bsz), budget = 226 * 1024;
+    const int l3p = profs[P.prof][2], d3 = 2 * l3p + 1, warps = src_warps_for(bsz);
+    const int budget = 226 * 1024 / ctas_per_sm_for(bsz);
     const int g = src_ring_g(bsz, P.CPL, l3p);
     auto base = [&](int chunk) { return (32 * 4 + 32 * P.KP * bsz + chunk * P.src_cy_stride * bsz + 15) / 16 * 16; };
     auto per_warp = [&](int chunk) { return base(chunk) + (2 * g * d3 * 32 * P.CPL * bsz + 15) / 16 * 16; };
@@ -404,10 +406,11 @@ int uvw_chunk_rows(const Plan& p, long long n_nodes, int dir) {
 }
 
 int uvu_src_slots(const Plan& p, long long n_nodes) {
-  // one wave of one-CTA-per-SM blocks, each serving one input-block tile
+  // one wave of source-pass CTAs, each serving one input-block tile
   const long long t = std::max<long long>(1, (long long)p.in_tiles.size());
-  const int w = src_warps_for(p.dtype == TP_F32 ? 4 : 8);
-  long long s = (long long)w * std::max<long long>(1, kSMs / t);
+  const int bsz = p.dtype == TP_F32 ? 4 : 8;
+  const int w = src_warps_for(bsz);
+  long long s = (long long)w * std::max<long long>(1, kSMs * ctas_per_sm_for(bsz) / t);
   s = std::min<long long>(s, std::max<long long>(1, n_nodes));
   return (int)s;
 }

@@ -10,23 +10,28 @@ constexpr int kWarpsPerBlock = 8; // warps per CTA of the warp-task kernels
 constexpr int kSMs = 148;         // streaming multiprocessors of a B200
 constexpr int kTnSplits = 8;      // split-K partial copies of A_bar in the uvw backward
 
-// Warps per CTA of the uvu source pass, which runs one CTA per SM: 16 for fp32,
-// 8 for fp64 (whose path bodies need more than 128 registers per thread).
+// Warps per CTA and CTAs per SM of the uvu source pass and forward: one CTA of
+// 16 warps for fp32; two CTAs of 4 warps for fp64 (whose path bodies need more
+// than 128 registers per thread), which spreads small graphs over twice the SMs.
 #ifdef __CUDACC__
 __host__ __device__
 #endif
-constexpr int src_warps_for(int scalar_bytes) { return scalar_bytes == 4 ? 16 : 8; }
+constexpr int src_warps_for(int scalar_bytes) { return scalar_bytes == 4 ? 16 : 4; }
+#ifdef __CUDACC__
+__host__ __device__
+#endif
+constexpr int ctas_per_sm_for(int scalar_bytes) { return scalar_bytes == 4 ? 1 : 2; }
 template <typename T>
 #ifdef __CUDACC__
 __host__ __device__
 #endif
 constexpr int src_warps() { return src_warps_for(sizeof(T)); }
 
-// Warps per CTA of the uvu forward, also one CTA per SM.
+// Warps per CTA of the uvu forward (CTAs per SM as for the source pass).
 #ifdef __CUDACC__
 __host__ __device__
 #endif
-constexpr int fwd_warps_for(int scalar_bytes) { return scalar_bytes == 4 ? 16 : 8; }
+constexpr int fwd_warps_for(int scalar_bytes) { return scalar_bytes == 4 ? 16 : 4; }
 template <typename T>
 #ifdef __CUDACC__
 __host__ __device__

@@ -434,7 +434,7 @@ __device__ __forceinline__ void src_tile(const UvuSrcParams<T>& p, const TileD& 
 }
 
 template <typename T, int KP, int CPL, class PR>
-__global__ void __launch_bounds__(src_warps<T>() * 32, 1)
+__global__ void __launch_bounds__(src_warps<T>() * 32, ctas_per_sm_for(sizeof(T)))
 uvu_src_kernel(const __grid_constant__ UvuSrcParams<T> p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   // every warp of a CTA serves the same input-block tile (one family of path

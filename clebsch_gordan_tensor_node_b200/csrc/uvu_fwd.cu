@@ -245,10 +245,10 @@ __device__ __forceinline__ void fwd_tile(const UvuFwdParams<T>& p, const TileD& 
   }
 }
 
-// One CTA per SM: 16 warps (fp32; a 128-register cap) or 8 (fp64), all of one
-// tile's path family at a time.
+// fp32: one CTA of 16 warps per SM (a 128-register cap); fp64: two CTAs of 4
+// warps. The warps of a CTA work on one tile's path family at a time.
 template <typename T, int KP, int CPL, int L1M, int L2M, int L3M>
-__global__ void __launch_bounds__(fwd_warps<T>() * 32, 1)
+__global__ void __launch_bounds__(fwd_warps<T>() * 32, ctas_per_sm_for(sizeof(T)))
 uvu_fwd_kernel(const __grid_constant__ UvuFwdParams<T> p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const long long task = (long long)blockIdx.x * fwd_warps<T>() + warp;
