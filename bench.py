@@ -250,7 +250,20 @@ def cpu_oracle_sample(cid: int, budget_s: float = 15.0):
         cores = os.cpu_count()
     return {"value": round(done_e / t_used, 1), "unit": "edges/s", "cores": cores, "kind": "oracle",
             "sample": f"forward of {n_recv} random receivers ({done_e} edges) of workload {cid}, "
-                      f"{t_used:.1f} s", "host_cpus": os.cpu_count()}
+                      f"{t_used:.1f} s", "host_cpus": os.cpu_count(), "workload_edges": len(wl.src)}
+
+
+# ----------------------------------------------------------------------------- ranks
+
+def aggregate_ranks(t_total_ms: float, n_edges: int, steps: int, world: int, dist=None, device="cpu"):
+    """Whole-job timing of N replicas: the max over ranks of the timed total
+    (ms), and the edges all ranks processed per second of that time."""
+    if dist is not None:
+        import torch
+        tt = torch.tensor([t_total_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_total_ms = float(tt.item())
+    return t_total_ms, n_edges * world * steps / (t_total_ms * 1e-3)
 
 
 # ----------------------------------------------------------------------------- main
@@ -268,8 +281,10 @@ def run_reference(args, rank, world):
         r = cpu_oracle_sample(args.config, budget_s=max(1.0, 20.0 / max(1, args.steps)))
         per_step.append(r["value"])
     val = statistics.median(per_step)
+    # a step of the workload at the sample's rate
+    ms_step = round(1e3 * r["workload_edges"] / val, 3)
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "edges/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": c.dtype, "data": "synthetic",
             "config": {"workload": c.name, "pass": "forward"},
             "cpu_baseline": {"value": val, "unit": "edges/s", "cores": r["cores"], "kind": "oracle",
@@ -298,13 +313,8 @@ def run_ours(args, rank, world, dist):
             bwd(d)
 
     times, clocks = time_steps(step, args.steps, args.warmup, flush, sampler, dist)
-    t_total = sum(times)
-    if dist is not None:
-        tt = torch.tensor([t_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_total = float(tt.item())
+    t_total, value = aggregate_ranks(sum(times), d["E"], args.steps, world, dist, dev)
     ms = t_total / args.steps
-    value = d["E"] * world * args.steps / (t_total * 1e-3)
     import clebsch_gordan_tensor_node_b200 as tpc
     assert tpc.tp_get_device_error() == 0
     res = {"metric": METRIC, "value": round(value, 1), "unit": "edges/s", "n_gpus": world,
