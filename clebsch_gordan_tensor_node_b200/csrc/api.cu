@@ -107,7 +107,6 @@ int forward_uvu(const Plan& P, const void* x, const void* Y, const void* phi, co
   prm.chunk = P.fwd_chunk;
   prm.warp_smem = P.fwd_warp_smem;
   prm.ring_off = P.fwd_ring_off;
-  prm.ring_g = P.fwd_ring_g;
   copy_tables(prm, P.out_tiles, P.paths_by_out);
   cudaError_t e = fwd_dispatch<T>(P, prm, s);
   return e == cudaSuccess ? TP_OK : cuda_fail(e, "uvu forward launch");

@@ -58,7 +58,7 @@ struct UvuFwdParams {
   int cy_stride;              // cY slots per staged edge (max over tiles, padded)
   int chunk;                  // edges staged per warp at a time (<= 32)
   int warp_smem;              // bytes of shared memory per warp
-  int ring_off, ring_g;       // x copy ring: byte offset in the warp's slice, edges per group
+  int ring_off;               // x copy ring: byte offset in the warp's slice
   TileD tiles[kMaxTiles];     // one per (output block, channel tile)
   PathD paths[kMaxPaths];     // grouped by output block
 };
@@ -84,7 +84,7 @@ struct UvuSrcParams {         // backward: source-owned grad_x, grad_A partials
   int cy_stride;              // cY slots per staged edge (max over tiles, padded)
   int chunk;                  // edges staged per warp at a time (<= 32)
   int warp_smem;              // bytes of shared memory per warp
-  int ring_off, ring_g;       // m_bar copy ring: byte offset in the warp's slice, edges per group
+  int ring_off;               // m_bar copy ring: byte offset in the warp's slice
   TileD tiles[kMaxTiles];     // one per (input block, channel tile)
   PathD paths[kMaxPaths];     // grouped by input block
 };

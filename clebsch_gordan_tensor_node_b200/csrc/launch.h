@@ -28,7 +28,6 @@ cudaError_t launch_uvu_src_for(const Plan& P, UvuSrcParams<T>& p, cudaStream_t s
   p.chunk = P.src_chunk;
   p.warp_smem = P.src_warp_smem;
   p.ring_off = P.src_ring_off;
-  p.ring_g = P.src_ring_g;
   if constexpr (std::is_same<T, float>::value) {
     if (P.CPL == 2) return P.KP == 8 ? launch_uvu_src<T, 8, 2>(p, P.prof, s) : launch_uvu_src<T, 16, 2>(p, P.prof, s);
   }

@@ -28,9 +28,9 @@ struct Plan {
   int edge_V = 1;           // channels per gather in the uvu backward edge pass
   int prof = 3;             // forward degree profile: 0 (2,2,2) 1 (1,3,3) 2 (3,3,3) 3 (4,4,4)
   int cy_stride = 0, fwd_chunk = 32, fwd_warp_smem = 0;
-  int fwd_ring_off = 0, fwd_ring_g = 1;   // forward: x copy ring offset (bytes) and group size
+  int fwd_ring_off = 0, fwd_ring_g = 1;   // forward: x copy ring offset (bytes); group size (= fwd_ring_g())
   int src_cy_stride = 0, src_chunk = 32, src_warp_smem = 0;
-  int src_ring_off = 0, src_ring_g = 1;   // source pass: m_bar copy ring offset (bytes) and group size
+  int src_ring_off = 0, src_ring_g = 1;   // source pass: m_bar ring offset (bytes); group size (= src_ring_g())
   std::vector<Block> bin, bout;
   std::vector<HostPath> paths;  // canonical enumeration order
   int c_in = 0, c_out = 0, dim_y = 0;

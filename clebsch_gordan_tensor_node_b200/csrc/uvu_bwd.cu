@@ -268,7 +268,7 @@ __device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& 
     }
   }
   // m_bar rows of the chunk's receivers go through a two-buffer ring of groups
-  // of ring_g edges: the copies of group g + 1 are in flight while group g is
+  // of G edges: the copies of group g + 1 are in flight while group g is
   // contracted. Each lane copies and later reads only its own channels.
   const T* gb = p.gout + pd.out_off + chl;
   const int mo = pd.mul_out, lane = threadIdx.x & 31;

@@ -38,7 +38,7 @@ struct FwdSmem {
   int* j;
   T* phi;
   T* cy;
-  T* ring;   // [2][ring_g][2 lmax_in + 1][32 CPL] x rows in flight
+  T* ring;   // [2][G][2 lmax_in + 1][32 CPL] x rows in flight (G = fwd_ring_g)
 };
 
 template <typename T, int KP>
