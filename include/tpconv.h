@@ -146,8 +146,9 @@ int tp_conv_launch_count(tp_plan_t plan, int64_t n_nodes, int pass, int* kernels
 /* Workspace bytes of tp_csr_build / tp_csr_transpose for n_nodes rows. */
 int tp_csr_workspace_size(int64_t n_nodes, size_t* bytes);
 
-/* Receiver CSR of a COO edge list (LunaTP §4.1; Sobek §4.5 "stable CSR
- * views"). Inputs (device): src[E], dst[E] with edge e = src[e] -> dst[e].
+/* Receiver CSR of a COO edge list (LunaTP §4.1; Sobek §4.5, which prepares a
+ * stable CSR before the kernels run). Inputs (device): src[E], dst[E] with
+ * edge e = src[e] -> dst[e].
  * Outputs (device): rowptr[N+1]; senders[E] = src of the edge at each CSR
  * position; perm[E] = COO index of the edge at each CSR position. Edges of one
  * receiver keep their input order. ws: device workspace of
@@ -158,7 +159,7 @@ int tp_csr_build(int64_t n_nodes, int64_t n_edges, const int32_t* src, const int
                  void* stream);
 
 /* Source view of a receiver CSR, for the node-feature gradient (LunaTP §4.4;
- * Sobek §4.3: "a separate source-contiguous CSR traversal owns x_bar").
+ * Sobek §4.3, where x_bar is owned by a second traversal grouped by sender).
  * Inputs (device): rowptr[N+1], senders[E] from tp_csr_build. Outputs
  * (device): colptr[N+1]; srcedge[E] = CSR positions grouped by sender, in
  * ascending order within a sender; srcrecv[E] = receiver of each of them. */

@@ -6,8 +6,8 @@
   (y, z, x) order, the symmetric traceless l=2 product);
 * equivariance of every real coupling under random rotations with real
   Wigner-D matrices fitted from spherical harmonics (pins the real basis
-  against the SH convention, LunaTP §2.1: "each path ... preserving
-  equivariance").
+  against the SH convention; LunaTP §2.1 requires every path to keep the
+  product equivariant).
 """
 import itertools
 
