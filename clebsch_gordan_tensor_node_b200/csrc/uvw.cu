@@ -351,31 +351,32 @@ __device__ __forceinline__ void edge_stage_compute(const UvwEdgeParams<T>& p, co
     for (int m = 0; m < D3; ++m) {
       const T cm = ct[m * 32];
       const T* sr = su + m * srow;
-      T acc = T(0);
+      T acc[4] = {T(0), T(0), T(0), T(0)};   // four independent chains over q
       if (p.vec) {
 #pragma unroll
         for (int q = 0; q < KP; q += VW) {
           if constexpr (VW == 4) {
             const float4 v = *reinterpret_cast<const float4*>(sr + q);
-            acc = fma(ph[q], v.x, acc); gphi[q] = fma(v.x, cm, gphi[q]);
-            acc = fma(ph[q + 1], v.y, acc); gphi[q + 1] = fma(v.y, cm, gphi[q + 1]);
-            acc = fma(ph[q + 2], v.z, acc); gphi[q + 2] = fma(v.z, cm, gphi[q + 2]);
-            acc = fma(ph[q + 3], v.w, acc); gphi[q + 3] = fma(v.w, cm, gphi[q + 3]);
+            acc[0] = fma(ph[q], v.x, acc[0]); gphi[q] = fma(v.x, cm, gphi[q]);
+            acc[1] = fma(ph[q + 1], v.y, acc[1]); gphi[q + 1] = fma(v.y, cm, gphi[q + 1]);
+            acc[2] = fma(ph[q + 2], v.z, acc[2]); gphi[q + 2] = fma(v.z, cm, gphi[q + 2]);
+            acc[3] = fma(ph[q + 3], v.w, acc[3]); gphi[q + 3] = fma(v.w, cm, gphi[q + 3]);
           } else {
             const double2 v = *reinterpret_cast<const double2*>(sr + q);
-            acc = fma(ph[q], v.x, acc); gphi[q] = fma(v.x, cm, gphi[q]);
-            acc = fma(ph[q + 1], v.y, acc); gphi[q + 1] = fma(v.y, cm, gphi[q + 1]);
+            acc[(q >> 1) & 2] = fma(ph[q], v.x, acc[(q >> 1) & 2]); gphi[q] = fma(v.x, cm, gphi[q]);
+            acc[((q >> 1) & 2) + 1] = fma(ph[q + 1], v.y, acc[((q >> 1) & 2) + 1]);
+            gphi[q + 1] = fma(v.y, cm, gphi[q + 1]);
           }
         }
       } else {
 #pragma unroll
         for (int q = 0; q < KP; ++q) {
           const T v = q < p.K ? sr[q] : T(0);
-          acc = fma(ph[q], v, acc);
+          acc[q & 3] = fma(ph[q], v, acc[q & 3]);
           gphi[q] = fma(v, cm, gphi[q]);
         }
       }
-      ct[m * 32] = acc;
+      ct[m * 32] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
     }
     T tb[D3];
 #pragma unroll
