@@ -502,8 +502,9 @@ int tp_conv_launch_count(tp_plan_t plan, int64_t n_nodes, int pass, int* kernels
   const long long gin = ((long long)P.uvw_in.size() + kMaxGemmBatch - 1) / kMaxGemmBatch;
   if (pass == 0)
     *kernels = (int)(1 + cr * (1 + gout));                       // pack A; per chunk: state, mixing
-  else
-    *kernels = (int)(1 + cr * (1 + 2 * gout + 1) + cs * (1 + gin) + 1);
+  else   // pack A; per receiver chunk: state, A_bar partials, their sum, S_bar, edge pass;
+         // per source chunk: source-view state, mixing; unpack A_bar
+    *kernels = (int)(1 + cr * (1 + gout + 1 + gout + 1) + cs * (1 + gin) + 1);
   return TP_OK;
 }
 

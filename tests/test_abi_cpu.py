@@ -89,3 +89,16 @@ def test_plan_errors(args, status):
     with pytest.raises(tpc.TpConvError) as ei:
         tpc.Plan(*args)
     assert ei.value.status == status
+
+
+def test_launch_count_matches_the_schedule():
+    """Kernels one call enqueues: uvu forward 1, backward 3 (edge, source, slot
+    sum); uvw per receiver chunk 2 forward (state, mixing) and 5 backward."""
+    import clebsch_gordan_tensor_node_b200 as tpc
+    uvu = tpc.Plan("8x0e+8x1o", 1, "8x0e+8x1o", 8, "uvu", "f32")
+    assert uvu.launch_count(1000, 0) == 1 and uvu.launch_count(1000, 1) == 3
+    assert uvu.launch_count(0, 0) == 0
+    uvw = tpc.Plan("8x0e+8x1o", 1, "8x0e+8x1o", 8, "uvw", "f32")
+    # a graph small enough for one state chunk in each direction, one GEMM batch
+    assert uvw.launch_count(100, 0) == 1 + 2
+    assert uvw.launch_count(100, 1) == 1 + 5 + 2 + 1
