@@ -389,7 +389,7 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
     for (auto& b : P.uvw_out) P.uvw_tc = P.uvw_tc && b.mul_own <= 64 && b.dcols % 4 == 0;
     for (auto& b : P.uvw_in) P.uvw_tc = P.uvw_tc && b.mul_own <= 64 && b.dcols % 4 == 0;
     const size_t bsz2 = dtype == TP_F32 ? 4 : 8;
-    if ((size_t)std::max(P.s_row_elems, P.sa_row_elems) * bsz2 > kUvwChunkBytes) {
+    if ((size_t)std::max(P.s_row_elems, P.sa_row_elems) * bsz2 > P.state_budget) {
       msg = "one node's uvw state exceeds the state chunk budget";
       return TP_EUNSUPPORTED;
     }
@@ -400,7 +400,7 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
 int uvw_chunk_rows(const Plan& p, long long n_nodes, int dir) {
   const size_t b = p.dtype == TP_F32 ? 4 : 8;
   const long long per = std::max<long long>(1, (dir == 0 ? p.s_row_elems : p.sa_row_elems));
-  long long r = (long long)(kUvwChunkBytes / (per * b));
+  long long r = (long long)(p.state_budget / (per * b));
   r = std::max<long long>(1, std::min<long long>(r, std::max<long long>(1, n_nodes)));
   return (int)r;
 }
@@ -439,17 +439,22 @@ void work_model(const Plan& p, long long N, long long E, int pass, double& flops
   const double b = p.dtype == TP_F32 ? 4.0 : 8.0;
   double fwd = 0, bwd = 0;
   for (auto& h : p.paths) {
-    const double d3 = 2 * h.l3 + 1, nnz = h.nnz, K = p.K;
+    const double d1 = 2 * h.l1 + 1, d3 = 2 * h.l3 + 1, nnz = h.nnz, K = p.K;
     if (p.mode == TP_UVU) {
       const double C = h.mul_in;
       fwd += 2.0 * E * C * (K + nnz + d3);
       bwd += 2.0 * E * C * (3 * K + 3 * nnz + 2 * d3);
     } else {
+      // state S (Eqs. 32-33) and mixing m = S A (Eqs. 34-35); the backward
+      // recomputes S, forms A_bar = S^T m_bar and S_bar = m_bar A^T (Eq. 36),
+      // runs the edge pass (C, T_bar, phi_bar, Y_bar), and builds and mixes the
+      // source state of x_bar
       const double ci = h.mul_in, co = h.mul_out;
       const double e = E * (2 * ci * nnz + 2 * K * ci * d3);
       const double r = N * 2 * d3 * K * ci * co;
       fwd += e + r;
-      bwd += r + e + E * (4 * K * ci * d3 + 4 * ci * nnz);
+      bwd += e + 2 * r + E * (4 * K * ci * d3 + 4 * ci * nnz) + E * (2 * co * nnz + 2 * K * co * d1) +
+             N * 2 * d1 * K * co * ci;
     }
   }
   const double in_b = b * ((double)N * p.c_in + (double)E * p.dim_y + (double)E * p.K + (double)p.K * p.n_w);

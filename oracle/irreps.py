@@ -59,14 +59,3 @@ def block_view(row, b: Block):
     """View the scalars of block b in an ir_mul row (or rows) as [..., 2l+1, mul]."""
     seg = row[..., b.offset:b.offset + b.size]
     return seg.reshape(seg.shape[:-1] + (b.dim, b.mul))
-
-
-def mul_ir_to_ir_mul(x, blocks: List[Block]):
-    """Convert a [..., C_x] mul_ir row (e3nn default: [u][m] per block) to ir_mul."""
-    import numpy as np
-    out = np.empty_like(x)
-    for b in blocks:
-        seg = x[..., b.offset:b.offset + b.size].reshape(x.shape[:-1] + (b.mul, b.dim))
-        out[..., b.offset:b.offset + b.size] = np.swapaxes(seg, -1, -2).reshape(
-            x.shape[:-1] + (b.size,))
-    return out

@@ -103,26 +103,38 @@ def concatenated_out_mul(irreps_in: str, sh, out_lp: Sequence[Tuple[int, int]]):
 
 
 def work_model(paths: List[Path], n_nodes: int, n_edges: int, K: int, mode: str) -> dict:
-    """Algorithmic flop counts (FMA = 2 flops) of the streamed schedule.
+    """Algorithmic flop counts (FMA = 2 flops) of the streamed schedules.
 
-    uvu (Sobek §3.1 order, w live only until consumed): per edge, channel, path:
-      K (w = phi . A) + nnz (CG contraction) + (2 l3 + 1) (weighted accumulate).
-    uvw (Sobek §4.2, Eqs. 32-35): per edge, path: 2 C_in nnz (Eq. 32) +
-      2 K C_in (2 l3 + 1) (Eq. 33); per receiver, path: 2 (2 l3 + 1) K C_in C_out
-      (Eq. 34-35).
+    uvu (Sobek §3.1 order, w live only until consumed), per edge, channel, path:
+      forward  K (w = phi . A) + nnz (CG contraction) + (2 l3 + 1) (weighted
+               accumulate);
+      backward 3 K (w, phi_bar, A_bar) + 3 nnz (h, x_bar, Y_bar contractions)
+               + 2 (2 l3 + 1).
+    uvw (Sobek §4.2 Eqs. 32-35 forward, §4.3 backward), per path with
+    d1 = 2 l1 + 1, d3 = 2 l3 + 1:
+      state  e  = E (2 C_in nnz + 2 K C_in d3)        (Eqs. 32-33)
+      mixing r  = N 2 d3 K C_in C_out                 (Eqs. 34-35)
+      forward  = e + r;
+      backward = e (state recomputed) + 2 r (A_bar = S^T m_bar and
+               S_bar = m_bar A^T, Eq. 36) + E (4 K C_in d3 + 4 C_in nnz) (edge
+               pass: C, T_bar, phi_bar, Y_bar) + E (2 C_out nnz + 2 K C_out d1)
+               (source state of x_bar) + N 2 d1 K C_out C_in (its mixing).
     """
     fwd = 0
     bwd = 0
     for p in paths:
         nnz = len(real_cg_sparse(p.l1, p.l2, p.l3))
+        d1 = 2 * p.l1 + 1
         d3 = 2 * p.l3 + 1
         if mode == "uvu":
             C = p.mul_in
             fwd += 2 * n_edges * C * (K + nnz + d3)
             bwd += 2 * n_edges * C * (3 * K + 3 * nnz + 2 * d3)
         else:
-            e = n_edges * (2 * p.mul_in * nnz + 2 * K * p.mul_in * d3)
-            r = n_nodes * 2 * d3 * K * p.mul_in * p.mul_out
+            ci, co = p.mul_in, p.mul_out
+            e = n_edges * (2 * ci * nnz + 2 * K * ci * d3)
+            r = n_nodes * 2 * d3 * K * ci * co
             fwd += e + r
-            bwd += r + e + n_edges * (4 * K * p.mul_in * d3 + 4 * p.mul_in * nnz)
+            bwd += (e + 2 * r + n_edges * (4 * K * ci * d3 + 4 * ci * nnz)
+                    + n_edges * (2 * co * nnz + 2 * K * co * d1) + n_nodes * 2 * d1 * K * co * ci)
     return {"fwd_flops": fwd, "bwd_flops": bwd}
