@@ -60,6 +60,7 @@ class Plan:
         self.info = info
         self.c_in, self.c_out, self.dim_y = info.c_in, info.c_out, info.dim_y
         self.n_radial, self.n_paths, self.n_w = info.n_radial, info.n_paths, info.n_w
+        self.state_budget = 1 << 30
 
     @property
     def handle(self):
@@ -84,6 +85,11 @@ class Plan:
         c = (ctypes.c_double * n)()
         check(lib().tp_conv_plan_cg(self._h, index, m1, m2, m3, c, n), "tp_conv_plan_cg")
         return [(m1[k], m2[k], m3[k], c[k]) for k in range(n)]
+
+    def set_state_budget(self, nbytes: int) -> None:
+        """Bytes of one uvw receiver-state chunk (tp_conv_plan_set_state_budget)."""
+        check(lib().tp_conv_plan_set_state_budget(self._h, nbytes), "tp_conv_plan_set_state_budget")
+        self.state_budget = nbytes
 
     def workspace_size(self, n_nodes: int, pass_: int) -> int:
         out = ctypes.c_size_t()

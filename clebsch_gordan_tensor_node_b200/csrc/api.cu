@@ -467,6 +467,19 @@ int tp_conv_plan_cg(tp_plan_t plan, int index, int32_t* m1, int32_t* m2, int32_t
   return n;
 }
 
+int tp_conv_plan_set_state_budget(tp_plan_t plan, size_t bytes) {
+  if (!plan) return fail(TP_EINVAL, "NULL plan");
+  Plan& P = plan->p;
+  if (P.mode != TP_UVW) return TP_OK;
+  const size_t b = P.dtype == TP_F32 ? 4 : 8;
+  const size_t one = (size_t)std::max(P.s_row_elems, P.sa_row_elems) * b;
+  if (bytes < one)
+    return fail(TP_EINVAL, "state budget " + std::to_string(bytes) + " bytes is below one node's state (" +
+                               std::to_string(one) + " bytes)");
+  P.state_budget = bytes;
+  return TP_OK;
+}
+
 int tp_conv_work_model(tp_plan_t plan, int64_t n_nodes, int64_t n_edges, int pass, double* flops,
                        double* bytes) {
   if (!plan || !flops || !bytes) return fail(TP_EINVAL, "NULL argument");

@@ -20,6 +20,9 @@ struct HostPath {
   int nnz;
 };
 
+// Default bytes of one uvw state chunk (the scratch budget of Sobek App. B.2).
+constexpr size_t kUvwChunkBytes = size_t(1) << 30;
+
 struct Plan {
   int mode = 0;     // 0 uvu, 1 uvw
   int dtype = 0;    // 0 f32, 1 f64
@@ -50,10 +53,10 @@ struct Plan {
   long long s_row_elems = 0;        // state elements per receiver (S)
   long long sa_row_elems = 0;       // state elements per source (S')
   bool uvw_tc = false;              // channel mixing on the tensor cores (fp32)
+  size_t state_budget = kUvwChunkBytes;   // bytes of one uvw state chunk
 };
 
-// Bytes of one uvw state chunk (the scratch budget of Sobek App. B.2).
-constexpr size_t kUvwChunkBytes = size_t(1) << 30;
+
 // Owners per uvw state chunk for a problem of n_nodes nodes (dir 0: S, 1: S').
 int uvw_chunk_rows(const Plan& p, long long n_nodes, int dir);
 

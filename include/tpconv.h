@@ -126,6 +126,18 @@ int tp_conv_plan_path(tp_plan_t plan, int index, tp_path_info_t* info);
 int tp_conv_plan_cg(tp_plan_t plan, int index, int32_t* m1, int32_t* m2, int32_t* m3, double* c,
                     int capacity);
 
+/* Bytes of one receiver-state chunk of a fully connected (uvw) plan. The uvw
+ * path reduces each receiver's edges into a state S_i with no output-channel
+ * axis and mixes it once (Sobek §4.2, Eqs. 33-35); receivers are processed in
+ * ranges whose states fit this budget, so the workspace is bounded by it and
+ * not by the edge count (Sobek App. B.2, fixed scratch budget). Default 1 GiB.
+ * A smaller budget gives more, smaller receiver (and source) chunks: less
+ * workspace, more launches (tp_conv_launch_count reports them). Host only.
+ * Errors: TP_EINVAL if `bytes` is below the state of one node
+ * (the message gives that size). Channelwise (uvu) plans keep no state
+ * chunks and accept any value without effect. */
+int tp_conv_plan_set_state_budget(tp_plan_t plan, size_t bytes);
+
 /* Algorithmic work of one pass (0 forward, 1 backward) on N nodes and E
  * edges: flops (FMA = 2) of the streamed schedule and compulsory HBM bytes
  * (each input read once, each output written once). Host only. */
@@ -207,7 +219,11 @@ int tp_conv_backward(tp_plan_t plan, const void* x, const void* Y, const void* p
  * that first call before any stream capture. Every call on a device shares the
  * one array and leaves its contents behind (each call clears what it needs
  * first); calls that may overlap on the GPU -- different streams, or threads
- * without ordering -- race on it and give wrong results. */
+ * without ordering -- race on it and give wrong results. The looked-up address
+ * is kept for the life of the process (as is the error word's): do not use the
+ * library on a device after cudaDeviceReset. The TP_EWORKSPACE limit is a
+ * guard: within the planner's limits (at most 96 channel tiles and 192 paths)
+ * one slot of a channelwise plan stays below about 2 MiB. */
 int tp_conv_backward_noalloc(tp_plan_t plan, const void* x, const void* Y, const void* phi,
                              const void* A, const int32_t* rowptr, const int32_t* senders,
                              const int32_t* colptr, const int32_t* srcedge, const int32_t* srcrecv,

@@ -102,3 +102,22 @@ def test_launch_count_matches_the_schedule():
     # a graph small enough for one state chunk in each direction, one GEMM batch
     assert uvw.launch_count(100, 0) == 1 + 2
     assert uvw.launch_count(100, 1) == 1 + 5 + 2 + 1
+
+
+def test_state_budget_sets_chunks_and_workspace():
+    """A smaller uvw state budget gives more receiver chunks (more launches) and a
+    smaller workspace; a budget below one node's state is rejected."""
+    c = CONFIGS[5]
+    plan = tpc.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.K, c.mode, c.dtype)
+    N = 4000
+    big_ws, big_n = plan.workspace_size(N, 1), plan.launch_count(N, 1)
+    plan.set_state_budget(64 << 20)
+    assert plan.workspace_size(N, 1) < big_ws
+    assert plan.launch_count(N, 1) > big_n
+    assert plan.launch_count(N, 0) > 3
+    with pytest.raises(tpc.TpConvError) as ei:
+        plan.set_state_budget(1024)
+    assert ei.value.status == -1 and "one node" in str(ei.value)
+    uvu = tpc.Plan("8x0e", 0, "8x0e", 4, "uvu", "f32")
+    uvu.set_state_budget(1)            # no state chunks: accepted, no effect
+    assert uvu.workspace_size(10, 0) == 0
