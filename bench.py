@@ -2,18 +2,23 @@
 
 Metric: TP-conv edges/s (forward, and forward+backward where the workload has a
 backward) with the achieved fraction of the roofline. The headline line times
-the forward of the MACE-like channelwise fp32 workload (4096 atoms, ~131k
-edges, 128x0e+128x1o -> 128x(0e+1o+2e+3o), L_sh 3, K 8). A step is one
-forward over that batch with every input resident in HBM. The L2 (126 MB) is
-flushed between timed steps by writing a 256 MiB buffer outside the timed
-events, because this workload's inputs fit in L2.
+one forward + backward step of the large-graph channelwise fp32 workload (100k
+atoms, ~4M edges, 64x(0e+1o+2e) -> 64x(l <= 2, both parities), L_sh 2, K 8),
+the largest single-GPU workload, with every input resident in HBM. Its inputs
+(~1 GB) are larger than the L2 (126 MB); a 256 MiB write outside the timed events
+flushes the L2 between steps anyway.
+
+The same JSON line carries, under "workloads", the forward (and forward +
+backward) of every workload, the MACE-like forward among them; under
+"workspace", the measured device memory of one forward + backward at E/4, E/2
+and E edges on the two largest workloads.
 
 Multi-GPU: the operator has no exchange step for independent batches, so each
 rank runs its own replica (weak scaling) and rank 0 reports the max time over
 ranks. `--impl reference` times the CPU oracle on the host cores instead.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                       [--config C] [--no-extra] [--no-cpu-baseline]
+                       [--config C] [--pass fwd|fwdbwd] [--no-extra] [--no-cpu-baseline]
 """
 from __future__ import annotations
 
@@ -149,48 +154,83 @@ def bwd(d):
 
 
 def time_steps(step, steps: int, warmup: int, flush, sampler=None, dist=None):
-    """Per-step CUDA-event times (ms) on the current stream, L2 flushed in between."""
+    """Per-step CUDA-event times (ms) on the current stream, L2 flushed in
+    between. `step(marks)` may append events it records between its passes;
+    returns (step times, per-pass times, clocks)."""
     import torch
     for _ in range(warmup):
         flush()
-        step()
+        step([])
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     if sampler:
         sampler.start()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    for a, b in evs:
+    evs = []
+    for _ in range(steps):
         flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        marks = []
         a.record()
-        step()
+        step(marks)
         b.record()
+        evs.append((a, marks, b))
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    return [a.elapsed_time(b) for a, b in evs], clocks
+    totals = [a.elapsed_time(b) for a, _, b in evs]
+    passes = []
+    for a, marks, b in evs:
+        pts = [a] + marks + [b]
+        passes.append([pts[k].elapsed_time(pts[k + 1]) for k in range(len(pts) - 1)])
+    return totals, passes, clocks
 
 
-def roofline_fb(d, ms: float) -> dict:
+def roofline_step(d, ms_pass, both: bool) -> dict:
+    """Roofline of the timed step: algorithmic flops of every pass over the step
+    time, against the derived ALU peak of the dtype; the per-pass numbers use
+    the CUDA-event time of each pass (the forward is one kernel launch)."""
     f0, b0 = d["plan"].work_model(d["N"], d["E"], 0)
-    f1, b1 = d["plan"].work_model(d["N"], d["E"], 1)
+    ms = sum(ms_pass)
+    if both:
+        f1, b1 = d["plan"].work_model(d["N"], d["E"], 1)
+        flops, nbytes = f0 + f1, b0 + b1
+    else:
+        flops, nbytes = f0, b0
     r = roofline(d, 0, ms)
-    ach = (f0 + f1) / (ms * 1e-3) / 1e12
-    r.update({"achieved": round(ach, 3), "frac": round(ach / r["peak"], 4), "algorithmic_flops": f0 + f1,
-              "compulsory_bytes": b0 + b1})
+    ach = flops / (ms * 1e-3) / 1e12
+    key = (d["cfg"].id, "fwdbwd" if both else "fwd")
+    t = NCU_TRAFFIC.get(key)
+    r.update({"achieved": round(ach, 3), "frac": round(ach / r["peak"], 4), "algorithmic_flops": flops,
+              "compulsory_bytes": nbytes, "traffic": None, "traffic_source": None,
+              "hbm_frac_of_measured": None,
+              "kernel": ("one step = forward (uvu_fwd_kernel) + backward (uvu_edge_kernel, "
+                         "uvu_src_kernel, reduce_slots_kernel)") if both and d["cfg"].mode == "uvu" else
+                        "one step = " + ("forward + backward" if both else "forward") + " launches"})
+    if t is not None:
+        hbm = measured_hbm_gbs()
+        r["traffic"] = t[0]
+        r["traffic_source"] = f"{t[1]}: dram__bytes_read.sum + dram__bytes_write.sum, {t[2]}"
+        if hbm:
+            r["hbm_frac_of_measured"] = round(t[0] / (ms * 1e-3) / 1e9 / hbm, 4)
+    per = {"fwd": {"ms": round(ms_pass[0], 5),
+                   "achieved": round(f0 / (ms_pass[0] * 1e-3) / 1e12, 3)}}
+    per["fwd"]["frac"] = round(per["fwd"]["achieved"] / r["peak"], 4)
+    if both:
+        per["bwd"] = {"ms": round(ms_pass[1], 5), "achieved": round(f1 / (ms_pass[1] * 1e-3) / 1e12, 3)}
+        per["bwd"]["frac"] = round(per["bwd"]["achieved"] / r["peak"], 4)
+    r["passes"] = per
     return r
 
 
-# DRAM bytes (read + write) per launch of the kernel that a (workload, pass)
-# timing is dominated by, from one ncu capture of the current kernel (the
-# summary under profiles/ names the command); None where no capture of the
-# current kernel exists.
-NCU_TRAFFIC = {
-    (2, 0): (21_665_024 + 564_480, "uvu_fwd_kernel", "profiles/uvu_fwd_kernel_mace_4096.md"),
-}
+# DRAM bytes (read + write) per step (summed over the step's kernels) or per
+# launch of a single-kernel pass, from ncu captures of the current kernels (the
+# summaries under profiles/ give the commands); absent where no capture of the
+# current kernels exists.
+NCU_TRAFFIC = {}
 
 
 def roofline(d, pass_: int, ms: float) -> dict:
@@ -198,20 +238,11 @@ def roofline(d, pass_: int, ms: float) -> dict:
     dt = d["cfg"].dtype
     peak = alu_peak(dt)
     ach = flops / (ms * 1e-3) / 1e12
-    r = {"bound": "alu", "achieved": round(ach, 3), "peak": round(peak, 2), "unit": "TFLOP/s",
-         "frac": round(ach / peak, 4), "traffic": None,
-         "peak_source": f"derived: {SMS} SMs x {FP32_LANES if dt == 'f32' else FP64_LANES} "
-                        f"{'FP32' if dt == 'f32' else 'FP64'} FMA lanes x 2 x {MAX_MHZ:.0f} MHz",
-         "algorithmic_flops": flops, "compulsory_bytes": nbytes,
-         "hbm_frac_of_measured": None}
-    t = NCU_TRAFFIC.get((d["cfg"].id, pass_))
-    if t is not None:
-        hbm = measured_hbm_gbs()
-        r["traffic"] = t[0]
-        r["traffic_source"] = f"{t[1]}: dram__bytes_read.sum + dram__bytes_write.sum, {t[2]}"
-        if hbm:
-            r["hbm_frac_of_measured"] = round(t[0] / (ms * 1e-3) / 1e9 / hbm, 4)
-    return r
+    return {"bound": "alu", "achieved": round(ach, 3), "peak": round(peak, 2), "unit": "TFLOP/s",
+            "frac": round(ach / peak, 4), "traffic": None,
+            "peak_source": f"derived: {SMS} SMs x {FP32_LANES if dt == 'f32' else FP64_LANES} "
+                           f"{'FP32' if dt == 'f32' else 'FP64'} FMA lanes x 2 x {MAX_MHZ:.0f} MHz",
+            "algorithmic_flops": flops, "compulsory_bytes": nbytes}
 
 
 def measured_hbm_gbs():
@@ -224,33 +255,67 @@ def measured_hbm_gbs():
 
 # ----------------------------------------------------------------------------- CPU oracle
 
-def cpu_oracle_sample(cid: int, budget_s: float = 15.0):
-    """Oracle forward on a bounded receiver sample of the workload: edges/s on host cores."""
-    from inputs import CONFIGS, make_workload
-    from oracle import conv as oconv
-    c = CONFIGS[cid]
-    pr = oconv.Problem(c.irreps_in, c.sh_lmax, c.irreps_out, c.K, c.mode)
-    wl = make_workload(cid, pr.n_w)
-    rng = np.random.default_rng(0)
-    order = rng.permutation(wl.n_nodes)
-    done_e, t_used, n_recv = 0, 0.0, 0
-    chunk = 64
-    while t_used < budget_s and n_recv < wl.n_nodes:
-        recv = order[n_recv:n_recv + chunk]
-        sel = np.isin(wl.dst, recv)
-        t0 = time.perf_counter()
-        oconv.forward(pr, wl.x, wl.Y[sel], wl.phi[sel], wl.A, wl.src[sel], wl.dst[sel], wl.n_nodes)
-        t_used += time.perf_counter() - t0
-        done_e += int(sel.sum())
-        n_recv += len(recv)
+def _cores():
     try:
         from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:
-        cores = os.cpu_count()
-    return {"value": round(done_e / t_used, 1), "unit": "edges/s", "cores": cores, "kind": "oracle",
-            "sample": f"forward of {n_recv} random receivers ({done_e} edges) of workload {cid}, "
-                      f"{t_used:.1f} s", "host_cpus": os.cpu_count(), "workload_edges": len(wl.src)}
+        return os.cpu_count()
+
+
+class OracleSampler:
+    """The CPU oracle (forward, or forward + backward) on windows of receivers of
+    a workload: each call runs the oracle on the incoming edges of the next
+    `n_recv` receivers of a seeded permutation and returns (edges, seconds)."""
+
+    def __init__(self, cid: int, both: bool):
+        from inputs import CONFIGS, make_workload
+        from oracle import conv as oconv
+        self.oconv = oconv
+        c = CONFIGS[cid]
+        self.cid, self.both = cid, both and c.backward
+        self.pr = oconv.Problem(c.irreps_in, c.sh_lmax, c.irreps_out, c.K, c.mode)
+        self.wl = make_workload(cid, self.pr.n_w)
+        self.order = np.random.default_rng(0).permutation(self.wl.n_nodes)
+        self.pos = 0
+
+    def run(self, n_recv: int):
+        wl = self.wl
+        if self.pos + n_recv > wl.n_nodes:
+            self.pos = 0
+        recv = self.order[self.pos:self.pos + n_recv]
+        self.pos += n_recv
+        sel = np.isin(wl.dst, recv)
+        args = (wl.x, wl.Y[sel], wl.phi[sel], wl.A, wl.src[sel], wl.dst[sel])
+        t0 = time.perf_counter()
+        self.oconv.forward(self.pr, *args, wl.n_nodes)
+        if self.both:
+            self.oconv.backward(self.pr, *args, wl.grad_out, wl.n_nodes)
+        return int(sel.sum()), time.perf_counter() - t0
+
+    def calibrate(self, seconds: float) -> int:
+        """Receivers per window for about `seconds` of oracle work."""
+        self.run(16)                       # first call fills the oracle's CG caches
+        e, t = self.run(16)
+        return int(max(1, min(self.wl.n_nodes, 16 * seconds / max(t, 1e-3))))
+
+    def label(self):
+        return "forward + backward" if self.both else "forward"
+
+
+def cpu_oracle_sample(cid: int, both: bool, budget_s: float = 15.0):
+    """Oracle edges/s on the host cores over a bounded receiver sample."""
+    s = OracleSampler(cid, both)
+    n_recv = s.calibrate(2.0)
+    done_e, t_used, n_done = 0, 0.0, 0
+    while t_used < budget_s and n_done < s.wl.n_nodes:
+        e, t = s.run(n_recv)
+        done_e += e
+        t_used += t
+        n_done += n_recv
+    return {"value": round(done_e / t_used, 1), "unit": "edges/s", "cores": _cores(), "kind": "oracle",
+            "sample": f"{s.label()} of {n_done} random receivers ({done_e} edges) of workload {cid}, "
+                      f"{t_used:.1f} s", "host_cpus": os.cpu_count(), "workload_edges": len(s.wl.src)}
 
 
 # ----------------------------------------------------------------------------- ranks
@@ -269,26 +334,34 @@ def aggregate_ranks(t_total_ms: float, n_edges: int, steps: int, world: int, dis
 # ----------------------------------------------------------------------------- main
 
 def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle as it stands, timed on the host cores.
+    Each step is the oracle on one window of receivers of the workload (sized
+    for about 1.5 s of work), so ms_per_step is the wall time of the work that
+    actually ran and value = edges of the windows / their time."""
     if rank != 0:
         return
     from inputs import CONFIGS
     c = CONFIGS[args.config]
-    per_step = []
+    both = args.pass_ == "fwdbwd" and c.backward
+    s = OracleSampler(args.config, both)
+    n_recv = s.calibrate(1.5)
     for _ in range(args.warmup):
-        cpu_oracle_sample(args.config, budget_s=1.0)
-    edges = 0
+        s.run(n_recv)
+    edges, secs = 0, 0.0
     for _ in range(args.steps):
-        r = cpu_oracle_sample(args.config, budget_s=max(1.0, 20.0 / max(1, args.steps)))
-        per_step.append(r["value"])
-    val = statistics.median(per_step)
-    # a step of the workload at the sample's rate
-    ms_step = round(1e3 * r["workload_edges"] / val, 3)
+        e, t = s.run(n_recv)
+        edges += e
+        secs += t
+    val = round(edges / secs, 1)
+    sample = (f"{s.label()} of {args.steps} windows of {n_recv} random receivers ({edges} edges in all) "
+              f"of the {len(s.wl.src)}-edge workload, {secs:.1f} s")
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "edges/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": c.dtype, "data": "synthetic",
-            "config": {"workload": c.name, "pass": "forward"},
-            "cpu_baseline": {"value": val, "unit": "edges/s", "cores": r["cores"], "kind": "oracle",
-                             "sample": r["sample"]},
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": c.name, "pass": s.label(), "sample": sample,
+                       "step": f"the oracle on one window of {n_recv} receivers"},
+            "cpu_baseline": {"value": val, "unit": "edges/s", "cores": _cores(), "kind": "oracle",
+                             "sample": sample},
             "e2e": {"value": val, "unit": "edges/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -305,16 +378,20 @@ def run_ours(args, rank, world, dist):
     d = setup(args.config, dev)
     c = d["cfg"]
     sampler = ClockSampler() if rank == 0 else None
-    both = args.pass_ == "fwdbwd"
+    both = args.pass_ == "fwdbwd" and c.backward
 
-    def step():
+    def step(marks):
         fwd(d)
         if both:
+            ev = torch.cuda.Event(enable_timing=True)
+            ev.record()
+            marks.append(ev)
             bwd(d)
 
-    times, clocks = time_steps(step, args.steps, args.warmup, flush, sampler, dist)
+    times, passes, clocks = time_steps(step, args.steps, args.warmup, flush, sampler, dist)
     t_total, value = aggregate_ranks(sum(times), d["E"], args.steps, world, dist, dev)
     ms = t_total / args.steps
+    ms_pass = [statistics.fmean(p[k] for p in passes) for k in range(len(passes[0]))]
     import clebsch_gordan_tensor_node_b200 as tpc
     assert tpc.tp_get_device_error() == 0
     res = {"metric": METRIC, "value": round(value, 1), "unit": "edges/s", "n_gpus": world,
@@ -325,35 +402,50 @@ def run_ours(args, rank, world, dist):
                       "n_nodes": d["N"], "n_edges": d["E"],
                       "irreps_in": c.irreps_in, "irreps_out": c.irreps_out, "sh_lmax": c.sh_lmax,
                       "n_radial": c.K, "mode": c.mode, "parallelism": f"replicas x{world}",
-                      "l2": "flushed between steps (256 MiB write outside the timed events)"},
+                      "l2": "inputs larger than L2; also flushed between steps (256 MiB write outside "
+                            "the timed events)"},
            "gpu_launches": args.steps * (d["plan"].launch_count(d["N"], 0)
                                          + (d["plan"].launch_count(d["N"], 1) if both else 0)),
-           "roofline": roofline(d, 0, ms) if not both else roofline_fb(d, ms), "clocks": clocks}
-    # end to end through the public API: pinned host inputs -> device -> forward -> host result
-    res["e2e"] = e2e(d, args, dev)
+           "roofline": roofline_step(d, ms_pass, both), "clocks": clocks}
+    # end to end through the public API: pinned host inputs -> device -> passes -> host results
+    res["e2e"] = e2e(d, args, both)
     if rank == 0 and not args.no_extra:
-        res["workloads"] = extra_workloads(args, dev, flush)
+        res["workloads"] = extra_workloads(args, dev, flush, d)
+        res["workspace"] = workspace_vs_edges(dev, d)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
-        res["cpu_baseline"] = cpu_oracle_sample(args.config)
+        res["cpu_baseline"] = cpu_oracle_sample(args.config, both)
     if rank == 0:
         print(json.dumps(res), flush=True)
 
 
-def e2e(d, args, dev):
+def e2e(d, args, both: bool):
+    """The metric through the public API with host buffers: every step copies
+    its inputs from pinned host memory, runs the passes and copies the results
+    (out, and the four gradients for forward + backward) back."""
     import torch
-    host = {k: d[k].cpu().pin_memory() for k in ("x", "Y", "phi", "A", "rowptr", "senders")}
-    devb = {k: torch.empty_like(d[k]) for k in host}
-    out_h = torch.empty(d["out"].shape, dtype=d["out"].dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_h.numel() * out_h.element_size()
+
     import clebsch_gordan_tensor_node_b200 as tpc
+    names = ["x", "Y", "phi", "A", "rowptr", "senders"]
+    if both:
+        names += ["colptr", "srcedge", "srcrecv", "gout"]
+    host = {k: d[k].cpu().pin_memory() for k in names}
+    devb = {k: torch.empty_like(d[k]) for k in host}
+    res_dev = [d["out"]] + (list(d["grads"]) if both else [])
+    res_host = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in res_dev]
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in res_host)
 
     def step():
         for k in host:
             devb[k].copy_(host[k], non_blocking=True)
-        o = tpc.tp_conv_forward(d["plan"], devb["x"], devb["Y"], devb["phi"], devb["A"], devb["rowptr"],
-                                devb["senders"], out=d["out"], ws=d["ws_f"])
-        out_h.copy_(o, non_blocking=True)
+        tpc.tp_conv_forward(d["plan"], devb["x"], devb["Y"], devb["phi"], devb["A"], devb["rowptr"],
+                            devb["senders"], out=d["out"], ws=d["ws_f"])
+        if both:
+            tpc.tp_conv_backward(d["plan"], devb["x"], devb["Y"], devb["phi"], devb["A"], devb["rowptr"],
+                                 devb["senders"], devb["colptr"], devb["srcedge"], devb["srcrecv"],
+                                 devb["gout"], out=d["grads"], ws=d["ws_b"])
+        for h, t in zip(res_host, res_dev):
+            h.copy_(t, non_blocking=True)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -367,52 +459,126 @@ def e2e(d, args, dev):
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / n
     return {"value": round(d["E"] / (ms * 1e-3), 1), "unit": "edges/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4)}
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4),
+            "pass": "forward+backward" if both else "forward"}
 
 
-def extra_workloads(args, dev, flush):
-    """Every workload's forward and (where defined) forward+backward."""
+def extra_workloads(args, dev, flush, head):
+    """Every workload's forward and (where defined) forward + backward."""
     import torch
 
     import clebsch_gordan_tensor_node_b200 as tpc
     out = {}
     for cid in (1, 2, 3, 4, 5):
         try:
-            d = setup(cid, dev)
+            d = head if cid == head["cfg"].id else setup(cid, dev)
         except tpc.TpConvError as e:
             out[str(cid)] = {"skipped": str(e)}
             continue
         try:
             k = 20 if d["E"] < 1_000_000 else 8
-            tf, _ = time_steps(lambda: fwd(d), k, 3, flush)
+            tf, _, _ = time_steps(lambda m: fwd(d), k, 3, flush)
             ms_f = statistics.median(tf)
+            rf = roofline_step(d, [ms_f], False)
             rec = {"workload": d["cfg"].name, "n_nodes": d["N"], "n_edges": d["E"], "dtype": d["cfg"].dtype,
                    "fwd_ms": round(ms_f, 5), "fwd_edges_per_s": round(d["E"] / (ms_f * 1e-3), 1),
-                   "fwd_roofline_frac": roofline(d, 0, ms_f)["frac"]}
+                   "fwd_roofline_frac": rf["frac"], "fwd_traffic": rf["traffic"],
+                   "gpu_launches_fwd": d["plan"].launch_count(d["N"], 0)}
             if d["cfg"].backward:
-                tb, _ = time_steps(lambda: bwd(d), k, 3, flush)
+                tb, _, _ = time_steps(lambda m: bwd(d), k, 3, flush)
                 ms_b = statistics.median(tb)
+                rb = roofline_step(d, [ms_f, ms_b], True)
                 rec.update({"bwd_ms": round(ms_b, 5),
                             "fwd_bwd_edges_per_s": round(d["E"] / ((ms_f + ms_b) * 1e-3), 1),
-                            "bwd_roofline_frac": roofline(d, 1, ms_b)["frac"],
-                            "workspace_bwd_bytes": d["plan"].workspace_size(d["N"], 1)})
+                            "bwd_roofline_frac": rb["passes"]["bwd"]["frac"],
+                            "fwd_bwd_roofline_frac": rb["frac"],
+                            "workspace_bwd_bytes": d["plan"].workspace_size(d["N"], 1),
+                            "gpu_launches_bwd": d["plan"].launch_count(d["N"], 1)})
             assert tpc.tp_get_device_error() == 0
             out[str(cid)] = rec
         except tpc.TpConvError as e:
             out[str(cid)] = {"skipped": str(e)}
-        del d
-        torch.cuda.empty_cache()
+        if d is not head:
+            del d
+            torch.cuda.empty_cache()
     return out
+
+
+def _edge_subset(d, keep: float, dev):
+    """The workload of `d` with a seeded fraction of its edges (same nodes)."""
+    import torch
+
+    import clebsch_gordan_tensor_node_b200 as tpc
+    wl = d["wl"]
+    m = np.random.default_rng(1000 + d["cfg"].id).random(len(wl.src)) < keep
+    src = torch.from_numpy(wl.src[m].astype(np.int32)).to(dev)
+    dst = torch.from_numpy(wl.dst[m].astype(np.int32)).to(dev)
+    N = d["N"]
+    rowptr, senders, perm = tpc.tp_csr_build(src, dst, N)
+    colptr, srcedge, srcrecv = tpc.tp_csr_transpose(rowptr, senders, N)
+    p = perm.long()
+    return dict(plan=d["plan"], N=N, E=int(m.sum()), x=d["x"], A=d["A"], gout=d["gout"], rowptr=rowptr,
+                senders=senders, colptr=colptr, srcedge=srcedge, srcrecv=srcrecv,
+                Y=torch.from_numpy(wl.Y[m]).to(dev)[p].contiguous(),
+                phi=torch.from_numpy(wl.phi[m]).to(dev)[p].contiguous())
+
+
+def workspace_vs_edges(dev, head):
+    """Device memory of one forward + backward through the public API at E/4,
+    E/2 and E edges (same nodes): the allocator's peak above what was allocated
+    before the calls (inputs and outputs preallocated, the binding allocates the
+    workspace), and the device memory taken outside the allocator."""
+    import torch
+
+    import clebsch_gordan_tensor_node_b200 as tpc
+    rec = {}
+    for cid in (4, 5):
+        d = head if cid == head["cfg"].id else setup(cid, dev)
+        row = {"workload": d["cfg"].name, "n_nodes": d["N"], "edges": [], "peak_bytes": [],
+               "outside_allocator_bytes": [], "workspace_size_fwd": d["plan"].workspace_size(d["N"], 0),
+               "workspace_size_bwd": d["plan"].workspace_size(d["N"], 1)}
+        for keep in (0.25, 0.5, 1.0):
+            s = _edge_subset(d, keep, dev)
+            out = torch.empty_like(d["out"])
+            grads = (torch.empty_like(s["x"]), torch.empty_like(s["Y"]), torch.empty_like(s["phi"]),
+                     torch.empty_like(s["A"]))
+
+            def step():
+                tpc.tp_conv_forward(s["plan"], s["x"], s["Y"], s["phi"], s["A"], s["rowptr"], s["senders"],
+                                    out=out)
+                tpc.tp_conv_backward(s["plan"], s["x"], s["Y"], s["phi"], s["A"], s["rowptr"], s["senders"],
+                                     s["colptr"], s["srcedge"], s["srcrecv"], s["gout"], out=grads)
+            step()
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+            torch.cuda.reset_peak_memory_stats()
+            base = torch.cuda.memory_allocated()
+            free0, res0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_reserved()
+            step()
+            torch.cuda.synchronize()
+            row["edges"].append(s["E"])
+            row["peak_bytes"].append(torch.cuda.max_memory_allocated() - base)
+            row["outside_allocator_bytes"].append(
+                (free0 - torch.cuda.mem_get_info()[0]) - (torch.cuda.memory_reserved() - res0))
+            assert tpc.tp_get_device_error() == 0
+            del s, out, grads
+            torch.cuda.empty_cache()
+        row["independent_of_edges"] = len(set(row["peak_bytes"])) == 1
+        rec[str(cid)] = row
+        if d is not head:
+            del d
+            torch.cuda.empty_cache()
+    return rec
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", type=int, default=2)
-    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "fwdbwd"])
+    ap.add_argument("--config", type=int, default=4)
+    ap.add_argument("--pass", dest="pass_", default="fwdbwd", choices=["fwd", "fwdbwd"])
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

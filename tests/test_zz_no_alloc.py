@@ -55,3 +55,21 @@ def test_noalloc_rejects_uvw_plans():
     z = ctypes.c_void_p(0)
     st = L.tp_conv_backward_noalloc(plan.handle, z, z, z, z, z, z, z, z, z, z, 1, 0, z, z, z, z, z)
     assert st == -2
+
+
+def test_noalloc_empty_graph_zeroes_grad_A():
+    """With no nodes there is nothing to accumulate: grad_A must still come back
+    zero (overwritten), whatever the previous calls left in the scratch."""
+    cid = 4
+    run = GpuRun(plan_for(cid), workload(cid, n_nodes=1500))
+    run.backward()                          # leave the scratch and outputs in use
+    L = _lib.lib()
+    gA = torch.full_like(run.A, float("nan"))
+    gx = torch.empty_like(run.x)
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    z = ctypes.c_void_p(0)
+    st = L.tp_conv_backward_noalloc(run.plan.handle, _p(run.x), z, z, _p(run.A), _p(run.rowptr), z,
+                                    _p(run.colptr), z, z, _p(run.gout), 0, 0, _p(gx), z, z, _p(gA), s)
+    assert st == 0, L.tp_last_error_message().decode()
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(gA).item() == 0 and torch.isfinite(gA).all()
