@@ -12,6 +12,9 @@ Test infrastructure. Definitions followed:
 * Sobek §3.2 / LunaTP Algorithm 2: h = <m_bar_i, T>, A_bar = sum phi h,
   phi_bar = sum A h, x_bar and Y_bar through the adjoints of the two partial
   Jacobians of the bilinear T, weighted by w.
+* Sobek §3.3 (Eqs. 23-31) / LunaTP Algorithm 3: the second-order program, the
+  product rule applied to w, T, m, h and the two operand adjoints along
+  directions (x_dot, Y_dot, phi_dot, A_dot).
 * Sobek §3.1 (streamed order, w live only until consumed) and §4.2 Eqs. 32-35
   (receiver state S, then m = S A) are written as separate loop nests, used only
   to check by brute force on tiny graphs that all orders agree.
@@ -139,6 +142,88 @@ def backward(pr: Problem, x, Y, phi, A, src, dst, grad_out, n_nodes: int, chunk:
         gphi[sl] = Wbar @ A.T
         np.add.at(gx, sc, gxc)
     return gx, gY, gphi, gA
+
+
+def double_backward(pr: Problem, x, Y, phi, A, src, dst, grad_out, dx, dY, dphi, dA, n_nodes: int,
+                    chunk: int = 65536):
+    """Second-order program of Sobek §3.3 (Eqs. 23-31), the directional
+    derivative of the forward output and of the four first-order adjoints along
+    (dx, dY, dphi, dA), with the output adjoint grad_out held fixed:
+
+      w_dot  = phi_dot A + phi A_dot                    T_dot = D_xT[x_dot] + D_YT[Y_dot]
+      m_dot  = sum (w_dot T + w T_dot)                  h_dot = <m_bar, T_dot>
+      A_bar_dot   = sum phi_dot h + phi h_dot           phi_bar_dot = A_dot h + A h_dot
+      x_bar_dot_j = sum w_dot B^x + w B^x_dot           Y_bar_dot   = sum w_dot B^Y + w B^Y_dot
+      with B^x = D_xT^* m_bar, B^Y = D_YT^* m_bar and their directional derivatives
+      (bilinearity: B^x_dot uses Y_dot, B^Y_dot uses x_dot).
+
+    This is also the product of the Hessian of <m_bar, m> with the direction and
+    the forward Jacobian applied to it, i.e. what LunaTP Algorithm 3 returns for
+    cotangents (dx, dY, dphi, dA) of the first-order outputs. Edge-chunked and
+    materialised like ``backward``. Returns (m_dot [N, C_out], x_bar_dot [N, C_x],
+    Y_bar_dot [E, dimY], phi_bar_dot [E, K], A_bar_dot [K, N_w]).
+    """
+    chunk = _chunk(pr, chunk)
+    f = lambda a: np.asarray(a, np.float64)
+    x, A, g, dx, dA = f(x), f(A), f(grad_out), f(dx), f(dA)
+    E = len(src)
+    mdot = np.zeros((n_nodes, pr.c_out))
+    gx = np.zeros((n_nodes, pr.c_in))
+    gY = np.zeros((E, pr.dim_y))
+    gphi = np.zeros((E, pr.K))
+    gA = np.zeros_like(A)
+    for s in range(0, E, chunk):
+        sl = slice(s, min(E, s + chunk))
+        sc, dc = src[sl], dst[sl]
+        Yc, pc, dYc, dpc = f(Y[sl]), f(phi[sl]), f(dY[sl]), f(dphi[sl])
+        W = pc @ A                                        # w
+        Wd = dpc @ A + pc @ dA                            # w_dot
+        Wbar = np.zeros_like(W)                           # h
+        Wbard = np.zeros_like(W)                          # h_dot
+        gi = g[dc]
+        Mc = np.zeros((len(sc), pr.c_out))
+        gxc = np.zeros((len(sc), pr.c_in))
+        for p in pr.paths:
+            b1, bo = pr.bin[p.i_in], pr.bout[p.i_out]
+            xj = _ir.block_view(x[sc], b1)
+            dxj = _ir.block_view(dx[sc], b1)
+            y0 = y_offset(p.l2)
+            Ye, dYe = Yc[:, y0:y0 + 2 * p.l2 + 1], dYc[:, y0:y0 + 2 * p.l2 + 1]
+            R = real_cg(p.l1, p.l2, p.l3)
+            T = _T(p, xj, Ye)
+            Td = _T(p, dxj, Ye) + _T(p, xj, dYe)           # T_dot
+            go = _ir.block_view(gi, bo)
+            Mo = _ir.block_view(Mc, bo)
+            Wp = W[:, p.w_off:p.w_off + p.n_w]
+            Wdp = Wd[:, p.w_off:p.w_off + p.n_w]
+            if pr.mode == "uvu":
+                Mo += Wdp[:, None, :] * T + Wp[:, None, :] * Td          # m_dot
+                h = np.einsum("ecu,ecu->eu", go, T)
+                hd = np.einsum("ecu,ecu->eu", go, Td)
+                wg = Wp[:, None, :] * go
+                wgd = Wdp[:, None, :] * go
+            else:
+                W3 = Wp.reshape(-1, p.mul_in, p.mul_out)
+                Wd3 = Wdp.reshape(-1, p.mul_in, p.mul_out)
+                Mo += np.einsum("euw,ecu->ecw", Wd3, T) + np.einsum("euw,ecu->ecw", W3, Td)
+                h = np.einsum("ecw,ecu->euw", go, T).reshape(len(sc), -1)
+                hd = np.einsum("ecw,ecu->euw", go, Td).reshape(len(sc), -1)
+                wg = np.einsum("euw,ecw->ecu", W3, go)
+                wgd = np.einsum("euw,ecw->ecu", Wd3, go)
+            Wbar[:, p.w_off:p.w_off + p.n_w] = h
+            Wbard[:, p.w_off:p.w_off + p.n_w] = hd
+            # x_bar_dot: w_dot D_xT^*(Y) m_bar + w D_xT^*(Y_dot) m_bar
+            bx = (np.einsum("abc,eb,ecu->eau", R, Ye, wgd, optimize=True)
+                  + np.einsum("abc,eb,ecu->eau", R, dYe, wg, optimize=True))
+            _ir.block_view(gxc, b1)[...] += bx
+            # Y_bar_dot: w_dot D_YT^*(x) m_bar + w D_YT^*(x_dot) m_bar
+            gY[sl, y0:y0 + 2 * p.l2 + 1] += (np.einsum("abc,eau,ecu->eb", R, xj, wgd, optimize=True)
+                                             + np.einsum("abc,eau,ecu->eb", R, dxj, wg, optimize=True))
+        gA += dpc.T @ Wbar + pc.T @ Wbard                 # A_bar_dot
+        gphi[sl] = Wbar @ dA.T + Wbard @ A.T              # phi_bar_dot
+        np.add.at(mdot, dc, Mc)
+        np.add.at(gx, sc, gxc)
+    return mdot, gx, gY, gphi, gA
 
 
 # ------------------------------------------------------------------ reassociated orders
