@@ -153,6 +153,21 @@ def bwd(d):
                                 ws=d["ws_b"])
 
 
+def dbl(d):
+    import clebsch_gordan_tensor_node_b200 as tpc
+    if "dirs" not in d:
+        import torch
+        g = torch.Generator(device=d["x"].device).manual_seed(3)
+        d["dirs"] = [torch.randn(d[k].shape, generator=g, device=d[k].device, dtype=d[k].dtype)
+                     for k in ("x", "Y", "phi", "A")]
+        d["dbl_out"] = (torch.empty_like(d["out"]),) + tuple(torch.empty_like(t) for t in d["grads"])
+        d["ws_d"] = torch.empty(max(1, d["plan"].workspace_size(d["N"], 2)), dtype=torch.uint8,
+                                device=d["x"].device)
+    return tpc.tp_conv_double_backward(d["plan"], d["x"], d["Y"], d["phi"], d["A"], d["rowptr"], d["senders"],
+                                       d["colptr"], d["srcedge"], d["srcrecv"], d["gout"], *d["dirs"],
+                                       out=d["dbl_out"], ws=d["ws_d"])
+
+
 def time_steps(step, steps: int, warmup: int, flush, sampler=None, dist=None):
     """Per-step CUDA-event times (ms) on the current stream, L2 flushed in
     between. `step(marks)` may append events it records between its passes;
@@ -494,6 +509,13 @@ def extra_workloads(args, dev, flush, head):
                             "fwd_bwd_roofline_frac": rb["frac"],
                             "workspace_bwd_bytes": d["plan"].workspace_size(d["N"], 1),
                             "gpu_launches_bwd": d["plan"].launch_count(d["N"], 1)})
+                if d["cfg"].mode == "uvu":
+                    td, _, _ = time_steps(lambda m: dbl(d), k, 3, flush)
+                    ms_d = statistics.median(td)
+                    fd, _ = d["plan"].work_model(d["N"], d["E"], 2)
+                    rec.update({"dbl_ms": round(ms_d, 5), "dbl_edges_per_s": round(d["E"] / (ms_d * 1e-3), 1),
+                                "dbl_roofline_frac": round(fd / (ms_d * 1e-3) / 1e12 / alu_peak(d["cfg"].dtype), 4),
+                                "gpu_launches_dbl": d["plan"].launch_count(d["N"], 2)})
             assert tpc.tp_get_device_error() == 0
             out[str(cid)] = rec
         except tpc.TpConvError as e:

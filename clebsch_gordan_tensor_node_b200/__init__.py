@@ -13,7 +13,8 @@ from typing import Optional, Tuple
 from ._lib import (TP_F32, TP_F64, TP_UVU, TP_UVW, PathInfo, PlanInfo, TpConvError, check, lib)
 
 __all__ = ["Plan", "tp_conv_plan", "tp_csr_build", "tp_csr_transpose", "tp_conv_forward",
-           "tp_conv_backward", "tp_conv_backward_noalloc", "tp_get_device_error", "TpConvError"]
+           "tp_conv_backward", "tp_conv_double_backward", "tp_conv_backward_noalloc", "tp_get_device_error",
+           "TpConvError"]
 
 
 def _torch():
@@ -204,6 +205,33 @@ def tp_conv_backward(plan: Plan, x, Y, phi, A, rowptr, senders, colptr, srcedge,
                                  _ptr(grad_out), N, E, _ptr(gx), _ptr(gY), _ptr(gphi), _ptr(gA),
                                  _ptr(ws), wsb, _stream(stream)), "tp_conv_backward")
     return gx, gY, gphi, gA
+
+
+def tp_conv_double_backward(plan: Plan, x, Y, phi, A, rowptr, senders, colptr, srcedge, srcrecv, grad_out,
+                            dx, dY, dphi, dA, out=None, ws=None, stream=None):
+    """Second-order program along (dx, dY, dphi, dA) with grad_out fixed.
+    Returns (d_out, dgrad_x, dgrad_Y, dgrad_phi, dgrad_A)."""
+    torch = _torch()
+    N, E = x.shape[0], senders.numel()
+    dt = plan.torch_dtype
+    _need(grad_out, dt, (N, plan.c_out), "grad_out")
+    _need(dx, dt, (N, plan.c_in), "dx")
+    _need(dY, dt, (E, plan.dim_y), "dY")
+    _need(dphi, dt, (E, plan.n_radial), "dphi")
+    _need(dA, dt, (plan.n_radial, plan.n_w), "dA")
+    if out is None:
+        out = (torch.empty(N, plan.c_out, dtype=dt, device=x.device),
+               torch.empty(N, plan.c_in, dtype=dt, device=x.device),
+               torch.empty(E, plan.dim_y, dtype=dt, device=x.device),
+               torch.empty(E, plan.n_radial, dtype=dt, device=x.device),
+               torch.empty(plan.n_radial, plan.n_w, dtype=dt, device=x.device))
+    ws, wsb = _workspace(plan.workspace_size(N, 2), x.device, ws)
+    check(lib().tp_conv_double_backward(plan.handle, _ptr(x), _ptr(Y), _ptr(phi), _ptr(A), _ptr(rowptr),
+                                        _ptr(senders), _ptr(colptr), _ptr(srcedge), _ptr(srcrecv),
+                                        _ptr(grad_out), _ptr(dx), _ptr(dY), _ptr(dphi), _ptr(dA), N, E,
+                                        *[_ptr(t) for t in out], _ptr(ws), wsb, _stream(stream)),
+          "tp_conv_double_backward")
+    return out
 
 
 def tp_conv_backward_noalloc(plan: Plan, x, Y, phi, A, rowptr, senders, colptr, srcedge, srcrecv,

@@ -52,6 +52,8 @@ SIGNATURES = {
     "tp_conv_backward": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_void_p,
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "tp_conv_double_backward": (c_int, [c_void_p] + [c_void_p] * 14 + [c_int64, c_int64] + [c_void_p] * 5
+                                + [c_void_p, c_size_t, c_void_p]),
     "tp_conv_backward_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                          c_void_p, c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_void_p,
                                          c_void_p, c_void_p, c_void_p, c_void_p]),

@@ -28,6 +28,7 @@ UNITS = {
     "uvu_fwd.cu": 9,
     "uvu_bwd.cu": 10,
     "uvw.cu": 10,
+    "uvu_dbwd.cu": 10,
     "gemm.cu": 1,
     "tc_gemm.cu": 1,
     "csr.cu": 1,

@@ -142,6 +142,44 @@ int backward_uvu(const Plan& P, const void* x, const void* Y, const void* phi, c
   return e == cudaSuccess ? TP_OK : cuda_fail(e, "grad_A reduction launch");
 }
 
+// Second-order program (Sobek §3.3): receiver, edge and source passes, then the
+// fixed-order sum of the A_bar_dot slot partials.
+template <typename T>
+int double_backward_uvu(const Plan& P, const void* const* in, const int* const* idx, const void* const* dir,
+                        int N, int E, void* const* out, void* ws, int* err, cudaStream_t s) {
+  UvuDbwdParams<T> p;
+  std::memset(&p, 0, sizeof(p));
+  p.x = (const T*)in[0]; p.Y = (const T*)in[1]; p.phi = (const T*)in[2]; p.A = (const T*)in[3];
+  p.gout = (const T*)in[4];
+  p.dx = (const T*)dir[0]; p.dY = (const T*)dir[1]; p.dphi = (const T*)dir[2]; p.dA = (const T*)dir[3];
+  p.rowptr = idx[0]; p.senders = idx[1]; p.colptr = idx[2]; p.srcedge = idx[3]; p.srcrecv = idx[4];
+  p.mdot = (T*)out[0]; p.gx = (T*)out[1]; p.gY = (T*)out[2]; p.gphi = (T*)out[3]; p.apart = (T*)ws;
+  p.err = err;
+  p.N = N; p.E = E; p.K = P.K; p.c_in = P.c_in; p.c_out = P.c_out; p.dim_y = P.dim_y; p.n_w = (int)P.n_w;
+  const bool k8 = P.KP == 8;
+  // receiver pass: m_dot
+  copy_tables(p, P.dbl_out_tiles, P.dbl_paths_by_out);
+  cudaError_t e = k8 ? launch_uvu_dbwd_recv<T, 8>(p, P.prof, s) : launch_uvu_dbwd_recv<T, 16>(p, P.prof, s);
+  if (e != cudaSuccess) return cuda_fail(e, "double backward receiver pass");
+  // edge pass: phi_bar_dot, Y_bar_dot
+  std::memset(p.paths, 0, sizeof(p.paths));
+  std::memcpy(p.paths, P.paths_canon.data(), P.paths_canon.size() * sizeof(PathD));
+  p.n_paths = (int)P.paths_canon.size();
+  constexpr int VW = std::is_same<T, float>::value ? 4 : 2;
+  if (P.edge_V == VW)
+    e = k8 ? launch_uvu_dbwd_edge<T, 8, VW>(p, P.prof, s) : launch_uvu_dbwd_edge<T, 16, VW>(p, P.prof, s);
+  else
+    e = k8 ? launch_uvu_dbwd_edge<T, 8, 1>(p, P.prof, s) : launch_uvu_dbwd_edge<T, 16, 1>(p, P.prof, s);
+  if (e != cudaSuccess) return cuda_fail(e, "double backward edge pass");
+  // source pass: x_bar_dot and the A_bar_dot slot partials, then their sum
+  copy_tables(p, P.dbl_in_tiles, P.dbl_paths_by_in);
+  p.n_slots = uvu_src_slots(P, N);
+  e = k8 ? launch_uvu_dbwd_src<T, 8>(p, P.prof, s) : launch_uvu_dbwd_src<T, 16>(p, P.prof, s);
+  if (e != cudaSuccess) return cuda_fail(e, "double backward source pass");
+  e = launch_reduce_slots<T>((const T*)ws, (T*)out[4], p.n_slots, (long long)P.K * P.n_w, s);
+  return e == cudaSuccess ? TP_OK : cuda_fail(e, "double backward A_bar reduction");
+}
+
 // ---------------------------------------------------------------- uvw
 
 bool use_tc(const Plan& P) { return P.uvw_tc; }
@@ -483,14 +521,14 @@ int tp_conv_plan_set_state_budget(tp_plan_t plan, size_t bytes) {
 int tp_conv_work_model(tp_plan_t plan, int64_t n_nodes, int64_t n_edges, int pass, double* flops,
                        double* bytes) {
   if (!plan || !flops || !bytes) return fail(TP_EINVAL, "NULL argument");
-  if (pass != 0 && pass != 1) return fail(TP_EINVAL, "pass must be 0 or 1");
+  if (pass < 0 || pass > 2) return fail(TP_EINVAL, "pass must be 0, 1 or 2");
   work_model(plan->p, n_nodes, n_edges, pass, *flops, *bytes);
   return TP_OK;
 }
 
 int tp_conv_workspace_size(tp_plan_t plan, int64_t n_nodes, int pass, size_t* bytes) {
   if (!plan || !bytes) return fail(TP_EINVAL, "NULL argument");
-  if (pass != 0 && pass != 1) return fail(TP_EINVAL, "pass must be 0 or 1");
+  if (pass < 0 || pass > 2) return fail(TP_EINVAL, "pass must be 0, 1 or 2");
   if (n_nodes < 0) return fail(TP_EINVAL, "negative node count");
   *bytes = workspace_bytes(plan->p, n_nodes, pass);
   return TP_OK;
@@ -498,7 +536,7 @@ int tp_conv_workspace_size(tp_plan_t plan, int64_t n_nodes, int pass, size_t* by
 
 int tp_conv_launch_count(tp_plan_t plan, int64_t n_nodes, int pass, int* kernels) {
   if (!plan || !kernels) return fail(TP_EINVAL, "NULL argument");
-  if (pass != 0 && pass != 1) return fail(TP_EINVAL, "pass must be 0 or 1");
+  if (pass < 0 || pass > 2) return fail(TP_EINVAL, "pass must be 0, 1 or 2");
   if (n_nodes < 0) return fail(TP_EINVAL, "negative node count");
   const Plan& P = plan->p;
   if (n_nodes == 0) {
@@ -506,7 +544,9 @@ int tp_conv_launch_count(tp_plan_t plan, int64_t n_nodes, int pass, int* kernels
     return TP_OK;
   }
   if (P.mode == TP_UVU) {
-    *kernels = pass == 0 ? 1 : 3;   // forward; edge pass, source pass, grad_A reduction
+    // forward; edge pass, source pass, grad_A reduction; receiver, edge and
+    // source passes of the second-order program and its A_bar reduction
+    *kernels = pass == 0 ? 1 : pass == 1 ? 3 : 4;
     return TP_OK;
   }
   const long long nr = uvw_chunk_rows(P, n_nodes, 0), ns = uvw_chunk_rows(P, n_nodes, 1);
@@ -621,6 +661,44 @@ int tp_conv_backward(tp_plan_t plan, const void* x, const void* Y, const void* p
                                    (int)n_nodes, (int)n_edges, grad_x, grad_Y, grad_phi, grad_A, ws, err, s)
              : backward_uvu<double>(P, x, Y, phi, A, rowptr, senders, colptr, srcedge, srcrecv, grad_out,
                                     (int)n_nodes, (int)n_edges, grad_x, grad_Y, grad_phi, grad_A, ws, err, s);
+}
+
+int tp_conv_double_backward(tp_plan_t plan, const void* x, const void* Y, const void* phi, const void* A,
+                            const int32_t* rowptr, const int32_t* senders, const int32_t* colptr,
+                            const int32_t* srcedge, const int32_t* srcrecv, const void* grad_out,
+                            const void* dx, const void* dY, const void* dphi, const void* dA, int64_t n_nodes,
+                            int64_t n_edges, void* d_out, void* dgrad_x, void* dgrad_Y, void* dgrad_phi,
+                            void* dgrad_A, void* ws, size_t ws_bytes, void* stream) {
+  if (!plan) return fail(TP_EINVAL, "NULL plan");
+  const Plan& P = plan->p;
+  int st = check_sizes(n_nodes, n_edges);
+  if (st) return st;
+  if (!x || !A || !rowptr || !colptr || !grad_out || !dx || !dA || !d_out || !dgrad_x || !dgrad_A ||
+      (n_edges > 0 && (!Y || !phi || !senders || !srcedge || !srcrecv || !dY || !dphi || !dgrad_Y || !dgrad_phi)))
+    return fail(TP_EINVAL, "NULL device pointer");
+  const void* f[] = {x, A, grad_out, dx, dA, d_out, dgrad_x, dgrad_A};
+  for (const void* q : f)
+    if (!al16(q)) return fail(TP_EINVAL, "floating-point buffers must be 16-byte aligned");
+  if (n_edges > 0 && (!al16(Y) || !al16(phi) || !al16(dY) || !al16(dphi) || !al16(dgrad_Y) || !al16(dgrad_phi)))
+    return fail(TP_EINVAL, "floating-point buffers must be 16-byte aligned");
+  if (P.mode == TP_UVW) return fail(TP_EUNSUPPORTED, "double backward of fully connected plans");
+  if (!P.dbl_ok) return fail(TP_EUNSUPPORTED, "double backward: more than 96 channel tiles of 32");
+  const size_t need = workspace_bytes(P, n_nodes, 2);
+  if (ws_bytes < need || (!ws && need > 0)) return fail(TP_EWORKSPACE, "workspace too small");
+  int* err = nullptr;
+  if ((st = error_word(&err))) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (n_nodes == 0) {
+    cudaError_t e = cudaMemsetAsync(dgrad_A, 0, (size_t)P.K * P.n_w * (P.dtype == TP_F32 ? 4 : 8), s);
+    return e == cudaSuccess ? TP_OK : cuda_fail(e, "memset dgrad_A");
+  }
+  const void* in[] = {x, Y, phi, A, grad_out};
+  const int* idx[] = {rowptr, senders, colptr, srcedge, srcrecv};
+  const void* dir[] = {dx, dY, dphi, dA};
+  void* out[] = {d_out, dgrad_x, dgrad_Y, dgrad_phi, dgrad_A};
+  return P.dtype == TP_F32
+             ? double_backward_uvu<float>(P, in, idx, dir, (int)n_nodes, (int)n_edges, out, ws, err, s)
+             : double_backward_uvu<double>(P, in, idx, dir, (int)n_nodes, (int)n_edges, out, ws, err, s);
 }
 
 int tp_get_device_error(void* stream) {

@@ -89,6 +89,25 @@ struct UvuSrcParams {         // backward: source-owned grad_x, grad_A partials
   PathD paths[kMaxPaths];     // grouped by input block
 };
 
+// Second-order program of the channelwise path (Sobek §3.3): directions
+// (dx, dY, dphi, dA) of the four inputs, the output adjoint gout held fixed.
+template <typename T>
+struct UvuDbwdParams {
+  const T* x; const T* Y; const T* phi; const T* A; const T* gout;
+  const T* dx; const T* dY; const T* dphi; const T* dA;
+  const int* rowptr; const int* senders;
+  const int* colptr; const int* srcedge; const int* srcrecv;
+  T* mdot;                    // receiver pass: directional output [N, C_out]
+  T* gY; T* gphi;             // edge pass: directional Y_bar [E, dimY], phi_bar [E, K]
+  T* gx; T* apart;            // source pass: directional x_bar [N, C_in]; A_bar slot partials
+  int* err;
+  int N, E, K, c_in, c_out, dim_y, n_w;
+  int n_paths, n_tiles, n_slots;
+  int split;                  // edge pass: warps sharing one group of 32 edges
+  TileD tiles[kMaxTiles];     // receiver pass: (output block, 32-channel tile); source pass: input blocks
+  PathD paths[kMaxPaths];     // receiver pass: by output block; source pass: by input block; edge pass: canonical
+};
+
 // ---- fully connected (uvw) path
 
 constexpr int kMaxBlocks = 32;

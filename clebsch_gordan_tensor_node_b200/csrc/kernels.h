@@ -21,6 +21,16 @@ cudaError_t launch_uvu_src(const UvuSrcParams<T>& p, int prof, cudaStream_t s);
 template <typename T>
 cudaError_t launch_reduce_slots(const T* part, T* out, int n_slots, long long n, cudaStream_t s);
 
+// second-order program of the channelwise path: receiver pass (m_dot), edge
+// pass (phi_bar_dot, Y_bar_dot; V channels per gather) and source pass
+// (x_bar_dot, A_bar_dot slot partials, zeroed first)
+template <typename T, int KP>
+cudaError_t launch_uvu_dbwd_recv(const UvuDbwdParams<T>& p, int prof, cudaStream_t s);
+template <typename T, int KP, int V>
+cudaError_t launch_uvu_dbwd_edge(const UvuDbwdParams<T>& p, int prof, cudaStream_t s);
+template <typename T, int KP>
+cudaError_t launch_uvu_dbwd_src(const UvuDbwdParams<T>& p, int prof, cudaStream_t s);
+
 template <typename T, int KP, int DIR>
 cudaError_t launch_uvw_sbuild_dir(const UvwSParams<T>& p, cudaStream_t s);
 

@@ -223,6 +223,9 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
   std::vector<TileD> unused;
   std::vector<Block> one{{1, 0, 1, 0}};
   add_tiles(one, all, P.paths, 1, unused, P.paths_canon);
+  add_tiles(P.bout, by_out, P.paths, 32, P.dbl_out_tiles, P.dbl_paths_by_out);
+  add_tiles(P.bin, by_in, P.paths, 32, P.dbl_in_tiles, P.dbl_paths_by_in);
+  P.dbl_ok = (int)P.dbl_out_tiles.size() <= kMaxTiles && (int)P.dbl_in_tiles.size() <= kMaxTiles;
   if ((int)P.out_tiles.size() > kMaxTiles || (int)P.in_tiles.size() > kMaxTiles) {
     msg = "more than " + std::to_string(kMaxTiles) + " channel tiles";
     return TP_EUNSUPPORTED;
@@ -419,7 +422,7 @@ size_t workspace_bytes(const Plan& p, long long n_nodes, int pass) {
   const size_t b = p.dtype == TP_F32 ? 4 : 8;
   size_t bytes = 0;
   if (p.mode == TP_UVU) {
-    if (pass == 1) bytes = (size_t)uvu_src_slots(p, n_nodes) * p.K * p.n_w * b;
+    if (pass >= 1) bytes = (size_t)uvu_src_slots(p, n_nodes) * p.K * p.n_w * b;
   } else {
     // packed A (forward operand; plus adjoint operand and packed A_bar in the
     // backward), each 256-byte aligned, and one (forward) or two (backward)
@@ -437,13 +440,17 @@ size_t workspace_bytes(const Plan& p, long long n_nodes, int pass) {
 
 void work_model(const Plan& p, long long N, long long E, int pass, double& flops, double& bytes) {
   const double b = p.dtype == TP_F32 ? 4.0 : 8.0;
-  double fwd = 0, bwd = 0;
+  double fwd = 0, bwd = 0, dbl = 0;
   for (auto& h : p.paths) {
     const double d1 = 2 * h.l1 + 1, d3 = 2 * h.l3 + 1, nnz = h.nnz, K = p.K;
     if (p.mode == TP_UVU) {
       const double C = h.mul_in;
       fwd += 2.0 * E * C * (K + nnz + d3);
       bwd += 2.0 * E * C * (3 * K + 3 * nnz + 2 * d3);
+      // second order: w, w_dot (3K); T, T_dot (3 nnz); m_dot (2 d3); h, h_dot
+      // (2 d3); A_bar_dot, phi_bar_dot (4K); x_bar_dot (2 nnz + 2 d1); Y_bar_dot
+      // (2 nnz)
+      dbl += 2.0 * E * C * (7 * K + 7 * nnz + 4 * d3 + 2 * d1);
     } else {
       // state S (Eqs. 32-33) and mixing m = S A (Eqs. 34-35); the backward
       // recomputes S, forms A_bar = S^T m_bar and S_bar = m_bar A^T (Eq. 36),
@@ -455,17 +462,28 @@ void work_model(const Plan& p, long long N, long long E, int pass, double& flops
       fwd += e + r;
       bwd += e + 2 * r + E * (4 * K * ci * d3 + 4 * ci * nnz) + E * (2 * co * nnz + 2 * K * co * d1) +
              N * 2 * d1 * K * co * ci;
+      // second order (Sobek §4.4): S and its directional state dS (C_dot, then
+      // phi_dot C + phi C_dot); dm = dS A + S dA, dA_bar = dS^T m_bar,
+      // S_bar = m_bar A^T, dS_bar = m_bar dA^T (5 mixing products); the edge pass
+      // on (S_bar, dS_bar, C, C_dot); the source state S' and dS', and
+      // x_bar_dot = dS' A' + S' dA'
+      dbl += e + E * (4 * ci * nnz + 4 * K * ci * d3) + 5 * r + E * (10 * K * ci * d3 + 10 * ci * nnz) +
+             E * (4 * co * nnz + 6 * K * co * d1) + 2 * N * 2 * d1 * K * co * ci;
     }
   }
   const double in_b = b * ((double)N * p.c_in + (double)E * p.dim_y + (double)E * p.K + (double)p.K * p.n_w);
   if (pass == 0) {
     flops = fwd;
     bytes = in_b + b * (double)N * p.c_out + 4.0 * E + 4.0 * (N + 1);
-  } else {
+  } else if (pass == 1) {
     flops = bwd;
     bytes = in_b + b * ((double)N * p.c_out + (double)N * p.c_in + (double)E * p.dim_y + (double)E * p.K +
                         (double)p.K * p.n_w) +
             12.0 * E + 8.0 * (N + 1);
+  } else {
+    // inputs and their directions, grad_out; m_dot and the four directional adjoints
+    flops = dbl;
+    bytes = 3 * in_b + b * 2.0 * (double)N * p.c_out + 12.0 * E + 8.0 * (N + 1);
   }
 }
 

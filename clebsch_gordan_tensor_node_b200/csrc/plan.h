@@ -44,6 +44,12 @@ struct Plan {
   std::vector<TileD> in_tiles;    // (input block, channel tile), paths_by_in ranges
   std::vector<PathD> paths_by_in;
   std::vector<PathD> paths_canon;
+  // second-order program: 32-channel tiles of the output and input blocks
+  std::vector<TileD> dbl_out_tiles;
+  std::vector<PathD> dbl_paths_by_out;
+  std::vector<TileD> dbl_in_tiles;
+  std::vector<PathD> dbl_paths_by_in;
+  bool dbl_ok = false;
   // fully connected (uvw) tables
   std::vector<UvwBlockD> uvw_out;   // output blocks, with paths_fwd ranges
   std::vector<PathD> paths_fwd;     // by output block; gathered = x block

@@ -138,19 +138,19 @@ int tp_conv_plan_cg(tp_plan_t plan, int index, int32_t* m1, int32_t* m2, int32_t
  * chunks and accept any value without effect. */
 int tp_conv_plan_set_state_budget(tp_plan_t plan, size_t bytes);
 
-/* Algorithmic work of one pass (0 forward, 1 backward) on N nodes and E
- * edges: flops (FMA = 2) of the streamed schedule and compulsory HBM bytes
- * (each input read once, each output written once). Host only. */
+/* Algorithmic work of one pass (0 forward, 1 backward, 2 double backward) on
+ * N nodes and E edges: flops (FMA = 2) of the streamed schedule and compulsory
+ * HBM bytes (each input read once, each output written once). Host only. */
 int tp_conv_work_model(tp_plan_t plan, int64_t n_nodes, int64_t n_edges, int pass, double* flops,
                        double* bytes);
 
-/* Workspace bytes that tp_conv_forward (pass 0) or tp_conv_backward (pass 1)
- * need for n_nodes receivers. It does not depend on the edge count (Sobek
+/* Workspace bytes that tp_conv_forward (pass 0), tp_conv_backward (pass 1) or
+ * tp_conv_double_backward (pass 2) need for n_nodes receivers. It does not depend on the edge count (Sobek
  * §3.4, Table 2: tensor-product workspace is bounded, not edge-sized). */
 int tp_conv_workspace_size(tp_plan_t plan, int64_t n_nodes, int pass, size_t* bytes);
 
-/* Number of kernels that one tp_conv_forward (pass 0) or tp_conv_backward
- * (pass 1) call enqueues for n_nodes receivers (memsets not counted). The
+/* Number of kernels that one tp_conv_forward (pass 0), tp_conv_backward
+ * (pass 1) or tp_conv_double_backward (pass 2) call enqueues for n_nodes receivers (memsets not counted). The
  * fully connected path works on receiver chunks of a fixed state budget, so
  * its count grows with n_nodes. Host only. */
 int tp_conv_launch_count(tp_plan_t plan, int64_t n_nodes, int pass, int* kernels);
@@ -201,6 +201,36 @@ int tp_conv_backward(tp_plan_t plan, const void* x, const void* Y, const void* p
                      const int32_t* srcedge, const int32_t* srcrecv, const void* grad_out,
                      int64_t n_nodes, int64_t n_edges, void* grad_x, void* grad_Y, void* grad_phi,
                      void* grad_A, void* ws, size_t ws_bytes, void* stream);
+
+/* Second-order program (Sobek §3.3 and §4.4; LunaTP Appendix F, Algorithm 3):
+ * the directional derivative, along v = (dx, dY, dphi, dA), of the forward
+ * output and of the four first-order adjoints, with grad_out held fixed:
+ *   d_out   = J v                 (J: Jacobian of the forward)
+ *   dgrad_* = H v                 (H: Hessian of <grad_out, forward>),
+ * per edge e = j -> i, path and channel (w = phi A, T = CG(x_j, Y_e)):
+ *   w_dot = dphi A + phi dA,  T_dot = CG(dx_j, Y_e) + CG(x_j, dY_e),
+ *   d_out_i += w_dot T + w T_dot,  h = <grad_out_i, T>,  h_dot = <grad_out_i, T_dot>,
+ *   dgrad_A += dphi h + phi h_dot,  dgrad_phi_e = dA h + A h_dot,
+ *   dgrad_x_j += w_dot D_xT^*(Y) grad_out_i + w D_xT^*(dY) grad_out_i,
+ *   dgrad_Y_e = w_dot D_YT^*(x) grad_out_i + w D_YT^*(dx) grad_out_i.
+ * For a loss L of the first-order outputs, passing v = (dL/dgrad_x, dL/dgrad_Y,
+ * dL/dgrad_phi, dL/dgrad_A) gives dL/d(x, Y, phi, A) in dgrad_* and dL/dgrad_out
+ * in d_out (the Hessian is symmetric), which is what a framework's double
+ * backward asks for. A direction of grad_out itself would add
+ * tp_conv_backward applied to it; callers add that separately.
+ * Inputs (device): x, Y, phi, A, grad_out and the CSR views as for
+ * tp_conv_backward; directions dx [N, C_in], dY [E, dimY], dphi [E, K] (CSR
+ * edge order), dA [K, N_w]. Outputs (device, overwritten): d_out [N, C_out],
+ * dgrad_x [N, C_in], dgrad_Y [E, dimY], dgrad_phi [E, K], dgrad_A [K, N_w].
+ * ws: at least tp_conv_workspace_size(plan, N, 2) bytes. Results are bitwise
+ * reproducible run to run (fixed ownership and order). Channelwise (uvu)
+ * plans; TP_EUNSUPPORTED for fully connected plans. */
+int tp_conv_double_backward(tp_plan_t plan, const void* x, const void* Y, const void* phi, const void* A,
+                            const int32_t* rowptr, const int32_t* senders, const int32_t* colptr,
+                            const int32_t* srcedge, const int32_t* srcrecv, const void* grad_out,
+                            const void* dx, const void* dY, const void* dphi, const void* dA, int64_t n_nodes,
+                            int64_t n_edges, void* d_out, void* dgrad_x, void* dgrad_Y, void* dgrad_phi,
+                            void* dgrad_A, void* ws, size_t ws_bytes, void* stream);
 
 /* tp_conv_backward for callers that cannot allocate device memory (no
  * counterpart in the pages: it is a service of this library). Plugins run from

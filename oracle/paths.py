@@ -119,9 +119,19 @@ def work_model(paths: List[Path], n_nodes: int, n_edges: int, K: int, mode: str)
                S_bar = m_bar A^T, Eq. 36) + E (4 K C_in d3 + 4 C_in nnz) (edge
                pass: C, T_bar, phi_bar, Y_bar) + E (2 C_out nnz + 2 K C_out d1)
                (source state of x_bar) + N 2 d1 K C_out C_in (its mixing).
+    Second order (Sobek §3.3 / §4.4), along (x_dot, Y_dot, phi_dot, A_dot):
+      uvu per edge, channel, path: w, w_dot (3 K); T, T_dot (3 nnz); m_dot
+          (2 d3); h, h_dot (2 d3); A_bar_dot, phi_bar_dot (4 K); x_bar_dot
+          (2 nnz + 2 d1); Y_bar_dot (2 nnz);
+      uvw: e + E (4 C_in nnz + 4 K C_in d3) (directional state dS) + 5 r (dm =
+          dS A + S dA, dA_bar = dS^T m_bar, S_bar, dS_bar = m_bar dA^T) +
+          E (10 K C_in d3 + 10 C_in nnz) (edge pass on S_bar, dS_bar, C, C_dot) +
+          E (4 C_out nnz + 6 K C_out d1) (source states S', dS') + 2 N 2 d1 K
+          C_out C_in (x_bar_dot = dS' A' + S' dA').
     """
     fwd = 0
     bwd = 0
+    dbl = 0
     for p in paths:
         nnz = len(real_cg_sparse(p.l1, p.l2, p.l3))
         d1 = 2 * p.l1 + 1
@@ -130,6 +140,7 @@ def work_model(paths: List[Path], n_nodes: int, n_edges: int, K: int, mode: str)
             C = p.mul_in
             fwd += 2 * n_edges * C * (K + nnz + d3)
             bwd += 2 * n_edges * C * (3 * K + 3 * nnz + 2 * d3)
+            dbl += 2 * n_edges * C * (7 * K + 7 * nnz + 4 * d3 + 2 * d1)
         else:
             ci, co = p.mul_in, p.mul_out
             e = n_edges * (2 * ci * nnz + 2 * K * ci * d3)
@@ -137,4 +148,7 @@ def work_model(paths: List[Path], n_nodes: int, n_edges: int, K: int, mode: str)
             fwd += e + r
             bwd += (e + 2 * r + n_edges * (4 * K * ci * d3 + 4 * ci * nnz)
                     + n_edges * (2 * co * nnz + 2 * K * co * d1) + n_nodes * 2 * d1 * K * co * ci)
-    return {"fwd_flops": fwd, "bwd_flops": bwd}
+            dbl += (e + n_edges * (4 * ci * nnz + 4 * K * ci * d3) + 5 * r
+                    + n_edges * (10 * K * ci * d3 + 10 * ci * nnz)
+                    + n_edges * (4 * co * nnz + 6 * K * co * d1) + 2 * n_nodes * 2 * d1 * K * co * ci)
+    return {"fwd_flops": fwd, "bwd_flops": bwd, "dbl_flops": dbl}

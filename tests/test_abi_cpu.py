@@ -66,6 +66,7 @@ def test_work_model_matches_oracle(cid):
     want = opaths.work_model(ps, N, E, c.K, c.mode)
     assert plan.work_model(N, E, 0)[0] == pytest.approx(want["fwd_flops"], rel=1e-12)
     assert plan.work_model(N, E, 1)[0] == pytest.approx(want["bwd_flops"], rel=1e-12)
+    assert plan.work_model(N, E, 2)[0] == pytest.approx(want["dbl_flops"], rel=1e-12)
 
 
 def test_workspace_does_not_depend_on_edges():

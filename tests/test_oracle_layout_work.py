@@ -107,6 +107,10 @@ def test_work_model_uvu_hand_count(K, N, E):
     wm = paths.work_model(ps, N, E, K, "uvu")
     assert wm["fwd_flops"] == 2 * E * (K + 6 + 3)
     assert wm["bwd_flops"] == 2 * E * (3 * K + 3 * 6 + 2 * 3)
+    # second order per edge and channel: w, w_dot (3K); T, T_dot (3 * 6); m_dot
+    # (2 * 3); h, h_dot (2 * 3); A_bar_dot, phi_bar_dot (4K); x_bar_dot (2 * 6 +
+    # 2 * 3); Y_bar_dot (2 * 6)
+    assert wm["dbl_flops"] == 2 * E * (7 * K + 7 * 6 + 4 * 3 + 2 * 3)
 
 
 def test_work_model_uvw_hand_count():
@@ -123,3 +127,8 @@ def test_work_model_uvw_hand_count():
     wm = paths.work_model(ps, 5, 10, 4, "uvw")
     assert wm["fwd_flops"] == 720 + 720
     assert wm["bwd_flops"] == 720 + 720 + 720 + 1440 + 1080 + 720
+    # second order: S 720; dS per edge 4*2*6 + 4*4*2*3 = 144 -> 1440; five
+    # mixing products 5 * 720; edge pass per edge 10*4*2*3 + 10*2*6 = 360 ->
+    # 3600; source states per edge 4*3*6 + 6*4*3*3 = 288 -> 2880; two source
+    # mixings 2 * 720
+    assert wm["dbl_flops"] == 720 + 1440 + 3600 + 3600 + 2880 + 1440
