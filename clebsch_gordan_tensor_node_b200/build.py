@@ -61,10 +61,25 @@ def _newest(paths):
     return max(os.path.getmtime(p) for p in paths)
 
 
+def _includes(path, found):
+    """Local headers a source includes, directly or through other headers."""
+    import re
+    try:
+        text = open(path).read()
+    except OSError:
+        return found
+    for name in re.findall(r'^\s*#\s*include\s+"([^"]+)"', text, re.M):
+        for d in (CSRC, INCLUDE, BUILD):
+            cand = os.path.join(d, name)
+            if os.path.exists(cand) and cand not in found:
+                found.add(cand)
+                _includes(cand, found)
+                break
+    return found
+
+
 def build(jobs: int | None = None, verbose: bool = False, force: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
-    headers = (glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh"))
-               + glob.glob(os.path.join(INCLUDE, "*.h")))
     # 1. compile-time CG table
     gen = os.path.join(BUILD, "cg_gen")
     table = os.path.join(BUILD, "cg_table.inc")
@@ -73,13 +88,13 @@ def build(jobs: int | None = None, verbose: bool = False, force: bool = False) -
     if force or not os.path.exists(table) or os.path.getmtime(table) < _newest(gen_src):
         _run(["g++", "-O2", "-std=c++17", "-o", gen, gen_src[0], gen_src[1]], verbose)
         _run([gen, str(CG_LMAX), table], verbose)
-    deps_time = _newest(headers + [table])
     # 2. objects
     nvcc = _nvcc()
     jobs_list = []
     for unit, nset in UNITS.items():
         src = os.path.join(CSRC, unit)
         stem = os.path.splitext(unit)[0]
+        deps_time = _newest([src] + sorted(_includes(src, set())))
         for k in range(nset):
             obj = os.path.join(BUILD, f"{stem}_{k}.o" if nset > 1 else f"{stem}.o")
             cmd = [nvcc, "-std=c++17", "-O3", "-lineinfo", *ARCH, "-Xcompiler", "-fPIC",
