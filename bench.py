@@ -509,13 +509,13 @@ def extra_workloads(args, dev, flush, head):
                             "fwd_bwd_roofline_frac": rb["frac"],
                             "workspace_bwd_bytes": d["plan"].workspace_size(d["N"], 1),
                             "gpu_launches_bwd": d["plan"].launch_count(d["N"], 1)})
-                if d["cfg"].mode == "uvu":
-                    td, _, _ = time_steps(lambda m: dbl(d), k, 3, flush)
-                    ms_d = statistics.median(td)
-                    fd, _ = d["plan"].work_model(d["N"], d["E"], 2)
-                    rec.update({"dbl_ms": round(ms_d, 5), "dbl_edges_per_s": round(d["E"] / (ms_d * 1e-3), 1),
-                                "dbl_roofline_frac": round(fd / (ms_d * 1e-3) / 1e12 / alu_peak(d["cfg"].dtype), 4),
-                                "gpu_launches_dbl": d["plan"].launch_count(d["N"], 2)})
+                td, _, _ = time_steps(lambda m: dbl(d), k, 3, flush)
+                ms_d = statistics.median(td)
+                fd, _ = d["plan"].work_model(d["N"], d["E"], 2)
+                rec.update({"dbl_ms": round(ms_d, 5), "dbl_edges_per_s": round(d["E"] / (ms_d * 1e-3), 1),
+                            "dbl_roofline_frac": round(fd / (ms_d * 1e-3) / 1e12 / alu_peak(d["cfg"].dtype), 4),
+                            "workspace_dbl_bytes": d["plan"].workspace_size(d["N"], 2),
+                            "gpu_launches_dbl": d["plan"].launch_count(d["N"], 2)})
             assert tpc.tp_get_device_error() == 0
             out[str(cid)] = rec
         except tpc.TpConvError as e:

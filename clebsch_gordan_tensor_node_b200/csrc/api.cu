@@ -201,13 +201,13 @@ void fill_blocks(UvwSParams<T>& p, const std::vector<UvwBlockD>& blocks, const s
 
 size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
-// m_g = S_g B_g for every output block of one receiver chunk (rows -> out).
+// m_g (+)= S_g B_g for every output block of one receiver chunk (rows -> out).
 // Tensor-core plans: Bf holds Bt_hi and Blo Bt_lo (transposed, split); the
 // SIMT GEMM reads Bf as B [D, N].
 template <typename T>
 cudaError_t mix_out(const Plan& P, const T* S, const T* Bf, const T* Blo, T* out, int r0, int nr, int nr_alloc,
                     const std::vector<UvwBlockD>& blocks, const std::vector<long long>& b_off, long long ld_out,
-                    int* err, cudaStream_t s) {
+                    int accumulate, int* err, cudaStream_t s) {
   if constexpr (std::is_same<T, float>::value) {
     if (use_tc(P)) {
       TcBatch tb;
@@ -226,7 +226,7 @@ cudaError_t mix_out(const Plan& P, const T* S, const T* Bf, const T* Blo, T* out
         }
         q.C = out;
         q.c = RowBlocked{r0, dc, ld_out, b.out_off, N};
-        q.M = M; q.N = N; q.D = D; q.pad = 0;
+        q.M = M; q.N = N; q.D = D; q.accumulate = accumulate;
         ++n;
         mm = std::max(mm, M);
         npmax = std::max(npmax, np);
@@ -251,11 +251,126 @@ cudaError_t mix_out(const Plan& P, const T* S, const T* Bf, const T* Blo, T* out
     q.G = nullptr;
     q.C = out;
     q.c = RowBlocked{r0, dc, ld_out, b.out_off, b.mul_own};
-    q.M = nr * dc; q.N = b.mul_own; q.D = b.dcols; q.accumulate = 0;
+    q.M = nr * dc; q.N = b.mul_own; q.D = b.dcols; q.accumulate = accumulate;
     mm = std::max(mm, q.M);
     mn = std::max(mn, q.N);
     if (n == kMaxGemmBatch || g + 1 == blocks.size()) {
       cudaError_t e = launch_gemm<T>(0, gb, n, mm, mn, s);
+      if (e != cudaSuccess) return e;
+      n = mm = mn = 0;
+    }
+  }
+  return cudaSuccess;
+}
+
+std::vector<long long> block_offsets(const std::vector<UvwBlockD>& blocks) {
+  std::vector<long long> off;
+  long long o = 0;
+  for (auto& g : blocks) {
+    off.push_back(o);
+    o += (long long)g.dcols * g.mul_own;
+  }
+  return off;
+}
+
+template <typename T>
+void state_params(UvwSParams<T>& sp, const Plan& P, const T* feat, const T* Y, const T* phi, const int* ptr,
+                  const int* nbr, const int* eid, T* S, int N, int E, int ld_feat, int nr_alloc,
+                  const std::vector<UvwBlockD>& blocks, const std::vector<PathD>& paths, int* err) {
+  sp.feat = feat; sp.Y = Y; sp.phi = phi;
+  sp.ptr = ptr; sp.nbr = nbr; sp.eid = eid; sp.S = S; sp.err = err;
+  sp.N = N; sp.E = E; sp.K = P.K; sp.ld_feat = ld_feat; sp.dim_y = P.dim_y; sp.n_feat_rows = N;
+  sp.r0 = 0; sp.nr = 0; sp.nr_alloc = nr_alloc; sp.accumulate = 0;
+  fill_blocks(sp, blocks, paths);
+}
+
+// The uvw edge pass's descriptor and shared-memory layout for one plan.
+template <typename T>
+int edge_params(const Plan& P, UvwEdgeParams<T>& ep, const T* x, const T* Y, const T* phi, const T* Sb,
+                const int* rowptr, const int* senders, T* gY, T* gphi, int N, int E, int NR, int* err) {
+  const size_t b = sizeof(T);
+  ep.x = x; ep.Y = Y; ep.phi = phi; ep.Sbar = Sb;
+  ep.rowptr = rowptr; ep.senders = senders; ep.gY = gY; ep.gphi = gphi; ep.err = err;
+  ep.N = N; ep.E = E; ep.K = P.K; ep.c_in = P.c_in; ep.dim_y = P.dim_y; ep.nr_alloc = NR;
+  ep.r0 = 0; ep.nr = 0; ep.accumulate = 0;
+  std::memset(ep.blocks, 0, sizeof(ep.blocks));
+  std::memset(ep.paths, 0, sizeof(ep.paths));
+  std::memcpy(ep.blocks, P.uvw_out.data(), P.uvw_out.size() * sizeof(UvwBlockD));
+  std::memcpy(ep.paths, P.paths_fwd.data(), P.paths_fwd.size() * sizeof(PathD));
+  ep.n_blocks = (int)P.uvw_out.size();
+  const int vw = 16 / (int)b;
+  bool vec = P.K == P.KP && P.c_in % vw == 0;
+  int xs = 0, sbar = 0;
+  for (const PathD& pd : P.paths_fwd) {
+    vec = vec && pd.x_off % vw == 0 && pd.mul_in % vw == 0;
+    const int nc = std::min(kEdgeTile, pd.mul_in);
+    xs = std::max(xs, 32 * edge_slot_stride((2 * pd.l1 + 1) * nc));
+    sbar = std::max(sbar, (2 * pd.l3 + 1) * nc * P.K);
+  }
+  for (size_t g = 0; g < P.uvw_out.size(); ++g)
+    for (int pi = P.uvw_out[g].pbeg; pi < P.uvw_out[g].pend; ++pi) ep.path_blk[pi] = (int8_t)g;
+  // the phi_bar partials [warps][K][32] reuse stage buffer 0 at the end of a round
+  xs = std::max(xs, kEdgeWarps * 32 * P.K - sbar);
+  ep.vec = vec ? 1 : 0;
+  ep.smem_sbar = (int)((sbar * b + 15) / 16 * 16);
+  ep.smem_stage = (int)((xs * b + 15) / 16 * 16) + ep.smem_sbar;
+  ep.smem_red = (int)((kEdgeWarps * 32 * P.dim_y * b + 15) / 16 * 16);
+  ep.smem_ct = (int)(kEdgeWarps * 32 * (2 * kLmax + 1) * b);
+  if (2 * (size_t)ep.smem_stage + ep.smem_red + ep.smem_ct + 32 * sizeof(int) > (size_t)227 * 1024)
+    return fail(TP_EUNSUPPORTED, "uvw edge pass: staging buffers exceed 227 KiB of shared memory");
+  return TP_OK;
+}
+
+template <typename T>
+cudaError_t edge_pass(const Plan& P, const UvwEdgeParams<T>& ep, cudaStream_t s) {
+  return P.KP == 8 ? launch_uvw_edge<T, 8>(ep, s) : launch_uvw_edge<T, 16>(ep, s);
+}
+
+// A_bar (+)= X_g^T m_bar_g over one receiver chunk (split-K partials, then their
+// fixed-order sum; accumulated over chunks when `acc`), X = S or dS.
+template <typename T>
+cudaError_t abar_chunk(const Plan& P, const T* X, const T* gout, T* Ab, T* Apart, size_t a_elems,
+                       const std::vector<long long>& bf_off, int r0, int nr, int NR, bool acc, cudaStream_t s) {
+  GemmBatch<T> gb;
+  int n = 0, mm = 0, mn = 0;
+  for (size_t g = 0; g < P.uvw_out.size(); ++g) {
+    const UvwBlockD& bd = P.uvw_out[g];
+    const int dc = 2 * bd.l + 1;
+    GemmProb<T>& q = gb.prob[n++];
+    q.G = gout;
+    q.g = RowBlocked{r0, dc, P.c_out, bd.out_off, bd.mul_own};
+    q.M = nr * dc; q.N = bd.mul_own; q.D = bd.dcols;
+    q.X = X + (size_t)NR * bd.s_off; q.B = nullptr; q.C = Ab + bf_off[g];
+    q.accumulate = acc;
+    mm = std::max(mm, q.D); mn = std::max(mn, q.N);
+    if (n == kMaxGemmBatch || g + 1 == P.uvw_out.size()) {
+      cudaError_t e = launch_gemm_tn_split<T>(gb, n, mm, mn, Ab, Apart, a_elems, kTnSplits, s);
+      if (e != cudaSuccess) return e;
+      n = mm = mn = 0;
+    }
+  }
+  return launch_sum_splits<T>(Apart, a_elems, kTnSplits, Ab, (long long)P.K * P.n_w, acc, s);
+}
+
+// S_bar_g = m_bar_g B_g^T over one receiver chunk (B packed from A or dA in
+// (u, q) row order).
+template <typename T>
+cudaError_t sbar_chunk(const Plan& P, const T* Buq, const T* gout, T* Sb, const std::vector<long long>& bf_off,
+                       int r0, int nr, int NR, cudaStream_t s) {
+  GemmBatch<T> gb;
+  int n = 0, mm = 0, mn = 0;
+  for (size_t g = 0; g < P.uvw_out.size(); ++g) {
+    const UvwBlockD& bd = P.uvw_out[g];
+    const int dc = 2 * bd.l + 1;
+    GemmProb<T>& q = gb.prob[n++];
+    q.G = gout;
+    q.g = RowBlocked{r0, dc, P.c_out, bd.out_off, bd.mul_own};
+    q.M = nr * dc; q.N = bd.mul_own; q.D = bd.dcols;
+    q.X = nullptr; q.B = Buq + bf_off[g]; q.C = Sb + (size_t)NR * bd.s_off;
+    q.accumulate = 0;
+    mm = std::max(mm, q.M); mn = std::max(mn, q.D);
+    if (n == kMaxGemmBatch || g + 1 == P.uvw_out.size()) {
+      cudaError_t e = launch_gemm_nt<T>(gb, n, mm, mn, s);
       if (e != cudaSuccess) return e;
       n = mm = mn = 0;
     }
@@ -275,26 +390,17 @@ int forward_uvw(const Plan& P, const void* x, const void* Y, const void* phi, co
   cudaError_t e = launch_pack_a<T>(P.pack, (const T*)A, tc ? nullptr : Bf, nullptr, tc ? Bf : nullptr, nullptr,
                                    Blo, nullptr, s);
   if (e != cudaSuccess) return cuda_fail(e, "pack A");
-  std::vector<long long> bf_off;
-  {
-    long long off = 0;
-    for (auto& g : P.uvw_out) {
-      bf_off.push_back(off);
-      off += (long long)g.dcols * g.mul_own;
-    }
-  }
-  UvwSParams<T> sp;
-  sp.feat = (const T*)x; sp.Y = (const T*)Y; sp.phi = (const T*)phi;
-  sp.ptr = rowptr; sp.nbr = senders; sp.eid = nullptr; sp.S = S; sp.err = err;
-  sp.N = N; sp.E = E; sp.K = P.K; sp.ld_feat = P.c_in; sp.dim_y = P.dim_y; sp.n_feat_rows = N;
-  fill_blocks(sp, P.uvw_out, P.paths_fwd);
+  const std::vector<long long> bf_off = block_offsets(P.uvw_out);
   const int NR = uvw_chunk_rows(P, N, 0);
-  sp.nr_alloc = NR;
+  UvwSParams<T> sp;
+  state_params(sp, P, (const T*)x, (const T*)Y, (const T*)phi, rowptr, senders, (const int*)nullptr, S, N, E,
+               P.c_in, NR, P.uvw_out, P.paths_fwd, err);
   for (int r0 = 0; r0 < N; r0 += NR) {
     sp.r0 = r0;
     sp.nr = std::min(NR, N - r0);
     if ((e = sbuild<T>(P, sp, 0, s)) != cudaSuccess) return cuda_fail(e, "uvw state build");
-    if ((e = mix_out<T>(P, S, Bf, Blo, (T*)out, r0, sp.nr, NR, P.uvw_out, bf_off, P.c_out, err, s)) != cudaSuccess)
+    if ((e = mix_out<T>(P, S, Bf, Blo, (T*)out, r0, sp.nr, NR, P.uvw_out, bf_off, P.c_out, 0, err, s)) !=
+        cudaSuccess)
       return cuda_fail(e, "uvw mixing");
   }
   return TP_OK;
@@ -324,114 +430,168 @@ int backward_uvw(const Plan& P, const void* x, const void* Y, const void* phi, c
   cudaError_t e = launch_pack_a<T>(pk, (const T*)A, Bf, tc ? nullptr : Ba, nullptr, tc ? Ba : nullptr, nullptr,
                                    Balo, s);
   if (e != cudaSuccess) return cuda_fail(e, "pack A");
-  std::vector<long long> bf_off, ba_off;
-  {
-    long long off = 0;
-    for (auto& g : P.uvw_out) {
-      bf_off.push_back(off);
-      off += (long long)g.dcols * g.mul_own;
-    }
-    off = 0;
-    for (auto& g : P.uvw_in) {
-      ba_off.push_back(off);
-      off += (long long)g.dcols * g.mul_own;
-    }
-  }
+  const std::vector<long long> bf_off = block_offsets(P.uvw_out), ba_off = block_offsets(P.uvw_in);
   // ---- receiver chunks: S, A_bar += S^T m_bar, S_bar = m_bar B^T, edge pass
   UvwSParams<T> sp;
-  sp.feat = (const T*)x; sp.Y = (const T*)Y; sp.phi = (const T*)phi;
-  sp.ptr = rowptr; sp.nbr = senders; sp.eid = nullptr; sp.S = S; sp.err = err;
-  sp.N = N; sp.E = E; sp.K = P.K; sp.ld_feat = P.c_in; sp.dim_y = P.dim_y; sp.n_feat_rows = N;
-  sp.nr_alloc = NR;
-  fill_blocks(sp, P.uvw_out, P.paths_fwd);
+  state_params(sp, P, (const T*)x, (const T*)Y, (const T*)phi, rowptr, senders, (const int*)nullptr, S, N, E,
+               P.c_in, NR, P.uvw_out, P.paths_fwd, err);
   UvwEdgeParams<T> ep;
-  ep.x = (const T*)x; ep.Y = (const T*)Y; ep.phi = (const T*)phi; ep.Sbar = Sb;
-  ep.rowptr = rowptr; ep.senders = senders; ep.gY = (T*)gY; ep.gphi = (T*)gphi; ep.err = err;
-  ep.N = N; ep.E = E; ep.K = P.K; ep.c_in = P.c_in; ep.dim_y = P.dim_y; ep.nr_alloc = NR;
-  std::memset(ep.blocks, 0, sizeof(ep.blocks));
-  std::memset(ep.paths, 0, sizeof(ep.paths));
-  std::memcpy(ep.blocks, P.uvw_out.data(), P.uvw_out.size() * sizeof(UvwBlockD));
-  std::memcpy(ep.paths, P.paths_fwd.data(), P.paths_fwd.size() * sizeof(PathD));
-  ep.n_blocks = (int)P.uvw_out.size();
-  {
-    const int vw = 16 / (int)b;
-    bool vec = P.K == P.KP && P.c_in % vw == 0;
-    int xs = 0, sbar = 0;
-    for (const PathD& pd : P.paths_fwd) {
-      vec = vec && pd.x_off % vw == 0 && pd.mul_in % vw == 0;
-      const int nc = std::min(kEdgeTile, pd.mul_in);
-      xs = std::max(xs, 32 * edge_slot_stride((2 * pd.l1 + 1) * nc));
-      sbar = std::max(sbar, (2 * pd.l3 + 1) * nc * P.K);
-    }
-    for (size_t g = 0; g < P.uvw_out.size(); ++g)
-      for (int pi = P.uvw_out[g].pbeg; pi < P.uvw_out[g].pend; ++pi) ep.path_blk[pi] = (int8_t)g;
-    // the phi_bar partials [warps][K][32] reuse stage buffer 0 at the end of a round
-    xs = std::max(xs, kEdgeWarps * 32 * P.K - sbar);
-    ep.vec = vec ? 1 : 0;
-    ep.smem_sbar = (int)((sbar * b + 15) / 16 * 16);
-    ep.smem_stage = (int)((xs * b + 15) / 16 * 16) + ep.smem_sbar;
-    ep.smem_red = (int)((kEdgeWarps * 32 * P.dim_y * b + 15) / 16 * 16);
-    ep.smem_ct = (int)(kEdgeWarps * 32 * (2 * kLmax + 1) * b);
-    if (2 * (size_t)ep.smem_stage + ep.smem_red + ep.smem_ct + 32 * sizeof(int) > (size_t)227 * 1024)
-      return fail(TP_EUNSUPPORTED, "uvw edge pass: staging buffers exceed 227 KiB of shared memory");
-  }
+  int st = edge_params(P, ep, (const T*)x, (const T*)Y, (const T*)phi, Sb, rowptr, senders, (T*)gY, (T*)gphi, N, E,
+                       NR, err);
+  if (st) return st;
   for (int r0 = 0; r0 < N; r0 += NR) {
     const int nr = std::min(NR, N - r0);
     sp.r0 = r0;
     sp.nr = nr;
     if ((e = sbuild<T>(P, sp, 0, s)) != cudaSuccess) return cuda_fail(e, "uvw state build");
-    for (int pass = 0; pass < 2; ++pass) {
-      GemmBatch<T> gb;
-      int n = 0, mm = 0, mn = 0;
-      for (size_t g = 0; g < P.uvw_out.size(); ++g) {
-        const UvwBlockD& bd = P.uvw_out[g];
-        const int dc = 2 * bd.l + 1;
-        GemmProb<T>& q = gb.prob[n++];
-        q.G = (const T*)gout;
-        q.g = RowBlocked{r0, dc, P.c_out, bd.out_off, bd.mul_own};
-        q.M = nr * dc; q.N = bd.mul_own; q.D = bd.dcols;
-        if (pass == 0) {            // A_bar_g (+)= S_g^T m_bar_g
-          q.X = S + (size_t)NR * bd.s_off; q.B = nullptr; q.C = Ab + bf_off[g];
-          q.accumulate = r0 > 0;
-          mm = std::max(mm, q.D); mn = std::max(mn, q.N);
-        } else {                    // S_bar_g = m_bar_g B_g^T
-          q.X = nullptr; q.B = Bf + bf_off[g]; q.C = Sb + (size_t)NR * bd.s_off;
-          q.accumulate = 0;
-          mm = std::max(mm, q.M); mn = std::max(mn, q.D);
-        }
-        if (n == kMaxGemmBatch || g + 1 == P.uvw_out.size()) {
-          e = pass == 0 ? launch_gemm_tn_split<T>(gb, n, mm, mn, Ab, Apart, a / b, kTnSplits, s)
-                        : launch_gemm_nt<T>(gb, n, mm, mn, s);
-          if (e != cudaSuccess) return cuda_fail(e, "uvw backward GEMM");
-          n = mm = mn = 0;
-        }
-      }
-      // A_bar (+)= the split partials, in split order
-      if (pass == 0 && (e = launch_sum_splits<T>(Apart, a / b, kTnSplits, Ab, (long long)P.K * P.n_w, r0 > 0, s)) !=
-                           cudaSuccess)
-        return cuda_fail(e, "uvw A_bar split sum");
-    }
+    if ((e = abar_chunk<T>(P, S, (const T*)gout, Ab, Apart, a / b, bf_off, r0, nr, NR, r0 > 0, s)) != cudaSuccess)
+      return cuda_fail(e, "uvw A_bar product");
+    if ((e = sbar_chunk<T>(P, Bf, (const T*)gout, Sb, bf_off, r0, nr, NR, s)) != cudaSuccess)
+      return cuda_fail(e, "uvw S_bar product");
     ep.r0 = r0;
     ep.nr = nr;
-    e = P.KP == 8 ? launch_uvw_edge<T, 8>(ep, s) : launch_uvw_edge<T, 16>(ep, s);
-    if (e != cudaSuccess) return cuda_fail(e, "uvw edge pass");
+    if ((e = edge_pass<T>(P, ep, s)) != cudaSuccess) return cuda_fail(e, "uvw edge pass");
   }
   // ---- source chunks: S' over the source view, x_bar = S' B'
   UvwSParams<T> ap;
-  ap.feat = (const T*)gout; ap.Y = (const T*)Y; ap.phi = (const T*)phi;
-  ap.ptr = colptr; ap.nbr = srcrecv; ap.eid = srcedge; ap.S = S; ap.err = err;
-  ap.N = N; ap.E = E; ap.K = P.K; ap.ld_feat = P.c_out; ap.dim_y = P.dim_y; ap.n_feat_rows = N;
-  ap.nr_alloc = NS;
-  fill_blocks(ap, P.uvw_in, P.paths_adj);
+  state_params(ap, P, (const T*)gout, (const T*)Y, (const T*)phi, colptr, srcrecv, srcedge, S, N, E, P.c_out, NS,
+               P.uvw_in, P.paths_adj, err);
   for (int s0r = 0; s0r < N; s0r += NS) {
     ap.r0 = s0r;
     ap.nr = std::min(NS, N - s0r);
     if ((e = sbuild<T>(P, ap, 1, s)) != cudaSuccess) return cuda_fail(e, "uvw source state build");
-    if ((e = mix_out<T>(P, S, Ba, Balo, (T*)gx, s0r, ap.nr, NS, P.uvw_in, ba_off, P.c_in, err, s)) != cudaSuccess)
+    if ((e = mix_out<T>(P, S, Ba, Balo, (T*)gx, s0r, ap.nr, NS, P.uvw_in, ba_off, P.c_in, 0, err, s)) !=
+        cudaSuccess)
       return cuda_fail(e, "uvw grad_x mixing");
   }
   e = launch_unpack_a<T>(P.pack, Ab, (T*)gA, s);
   return e == cudaSuccess ? TP_OK : cuda_fail(e, "unpack grad_A");
+}
+
+// The packed GEMM operands of one [K, N_w] weight tensor (A or its direction).
+template <typename T>
+struct PackedW {
+  T* fwd;      // forward mixing m = S B (tensor cores: B^T hi part)
+  T* fwd_lo;   // tensor cores: B^T lo part
+  T* adj;      // source mixing x_bar = S' B' (tensor cores: B'^T hi part)
+  T* adj_lo;
+  T* uq;       // S_bar = m_bar B^T, rows in (u, q) order
+};
+
+template <typename T>
+cudaError_t pack_w(const Plan& P, const T* W, PackedW<T>& o, char*& cur, size_t a, cudaStream_t s) {
+  const bool tc = use_tc(P);
+  auto take = [&]() {
+    T* p = (T*)cur;
+    cur += a;
+    return p;
+  };
+  o.uq = take();
+  o.fwd = take();
+  o.adj = take();
+  o.fwd_lo = tc ? take() : nullptr;
+  o.adj_lo = tc ? take() : nullptr;
+  UvwPackParams pk = P.pack;
+  pk.bf_uq = 1;
+  cudaError_t e = tc ? launch_pack_a<T>(pk, W, o.uq, nullptr, o.fwd, o.adj, o.fwd_lo, o.adj_lo, s)
+                     : launch_pack_a<T>(pk, W, o.uq, o.adj, nullptr, nullptr, nullptr, nullptr, s);
+  if (e != cudaSuccess || tc) return e;
+  pk.bf_uq = 0;
+  return launch_pack_a<T>(pk, W, o.fwd, nullptr, nullptr, nullptr, nullptr, nullptr, s);
+}
+
+// Second-order program of the fully connected path (Sobek §4.4), composed from
+// the first-order kernels by multilinearity: with the directional state
+// dS = S(dx, Y, phi) + S(x, dY, phi) + S(x, Y, dphi) per receiver chunk,
+//   m_dot       = dS A + S dA,             A_bar_dot = dS^T m_bar,
+//   phi_bar_dot = E_phi(dx, Y; S_bar) + E_phi(x, dY; S_bar) + E_phi(x, Y; dS_bar),
+//   Y_bar_dot   = E_Y(dx, phi; S_bar) + E_Y(x, dphi; S_bar) + E_Y(x, phi; dS_bar),
+// with S_bar = m_bar A^T, dS_bar = m_bar dA^T and E the edge pass (its phi_bar
+// does not read phi, its Y_bar does not read Y, so each call yields two wanted
+// terms); per source chunk x_bar_dot = (S'(dY, phi) + S'(Y, dphi)) A' + S' dA'.
+template <typename T>
+int double_backward_uvw(const Plan& P, const void* const* in, const int* const* idx, const void* const* dir, int N,
+                        int E, void* const* out, void* ws, int* err, cudaStream_t s) {
+  const size_t b = sizeof(T);
+  const size_t a = align256((size_t)P.K * P.n_w * b);
+  const T *x = (const T*)in[0], *Y = (const T*)in[1], *phi = (const T*)in[2], *A = (const T*)in[3],
+          *gout = (const T*)in[4];
+  const T *dx = (const T*)dir[0], *dY = (const T*)dir[1], *dphi = (const T*)dir[2], *dA = (const T*)dir[3];
+  const int *rowptr = idx[0], *senders = idx[1], *colptr = idx[2], *srcedge = idx[3], *srcrecv = idx[4];
+  T *mdot = (T*)out[0], *dgx = (T*)out[1], *dgY = (T*)out[2], *dgphi = (T*)out[3], *dgA = (T*)out[4];
+  char* cur = (char*)ws;
+  PackedW<T> pa, pd;
+  cudaError_t e = pack_w<T>(P, A, pa, cur, a, s);
+  if (e == cudaSuccess) e = pack_w<T>(P, dA, pd, cur, a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "pack A");
+  T* Ab = (T*)cur;
+  cur += a;
+  T* Apart = (T*)cur;
+  cur += kTnSplits * a;
+  const int NR = uvw_chunk_rows(P, N, 0), NS = uvw_chunk_rows(P, N, 1);
+  const size_t sm = std::max(align256((size_t)NR * P.s_row_elems * b), align256((size_t)NS * P.sa_row_elems * b));
+  T* S = (T*)cur;
+  T* Sb = (T*)(cur + sm);
+  const std::vector<long long> bf_off = block_offsets(P.uvw_out), ba_off = block_offsets(P.uvw_in);
+  UvwSParams<T> sp;
+  state_params(sp, P, x, Y, phi, rowptr, senders, (const int*)nullptr, S, N, E, P.c_in, NR, P.uvw_out, P.paths_fwd,
+               err);
+  UvwEdgeParams<T> ep;
+  int st = edge_params(P, ep, x, Y, phi, Sb, rowptr, senders, dgY, dgphi, N, E, NR, err);
+  if (st) return st;
+  auto build = [&](UvwSParams<T>& p, const T* feat, const T* y, const T* ph, int acc, int d) {
+    p.feat = feat; p.Y = y; p.phi = ph; p.accumulate = acc;
+    return sbuild<T>(P, p, d, s);
+  };
+  for (int r0 = 0; r0 < N; r0 += NR) {
+    const int nr = std::min(NR, N - r0);
+    sp.r0 = r0;
+    sp.nr = nr;
+    // directional state dS, then m_dot = dS A and A_bar_dot (+)= dS^T m_bar
+    if ((e = build(sp, dx, Y, phi, 0, 0)) != cudaSuccess || (e = build(sp, x, dY, phi, 1, 0)) != cudaSuccess ||
+        (e = build(sp, x, Y, dphi, 1, 0)) != cudaSuccess)
+      return cuda_fail(e, "uvw directional state");
+    if ((e = mix_out<T>(P, S, pa.fwd, pa.fwd_lo, mdot, r0, nr, NR, P.uvw_out, bf_off, P.c_out, 0, err, s)) !=
+        cudaSuccess)
+      return cuda_fail(e, "uvw directional mixing");
+    if ((e = abar_chunk<T>(P, S, gout, Ab, Apart, a / b, bf_off, r0, nr, NR, r0 > 0, s)) != cudaSuccess)
+      return cuda_fail(e, "uvw A_bar_dot product");
+    // primal state S, m_dot += S dA
+    if ((e = build(sp, x, Y, phi, 0, 0)) != cudaSuccess) return cuda_fail(e, "uvw state build");
+    if ((e = mix_out<T>(P, S, pd.fwd, pd.fwd_lo, mdot, r0, nr, NR, P.uvw_out, bf_off, P.c_out, 1, err, s)) !=
+        cudaSuccess)
+      return cuda_fail(e, "uvw mixing");
+    // edge pass on S_bar with (dx, Y, phi) and (x, dY, dphi), then on dS_bar
+    if ((e = sbar_chunk<T>(P, pa.uq, gout, Sb, bf_off, r0, nr, NR, s)) != cudaSuccess)
+      return cuda_fail(e, "uvw S_bar product");
+    ep.r0 = r0;
+    ep.nr = nr;
+    ep.x = dx; ep.Y = Y; ep.phi = phi; ep.accumulate = 0;
+    if ((e = edge_pass<T>(P, ep, s)) != cudaSuccess) return cuda_fail(e, "uvw edge pass");
+    ep.x = x; ep.Y = dY; ep.phi = dphi; ep.accumulate = 1;
+    if ((e = edge_pass<T>(P, ep, s)) != cudaSuccess) return cuda_fail(e, "uvw edge pass");
+    if ((e = sbar_chunk<T>(P, pd.uq, gout, Sb, bf_off, r0, nr, NR, s)) != cudaSuccess)
+      return cuda_fail(e, "uvw S_bar product");
+    ep.x = x; ep.Y = Y; ep.phi = phi; ep.accumulate = 1;
+    if ((e = edge_pass<T>(P, ep, s)) != cudaSuccess) return cuda_fail(e, "uvw edge pass");
+  }
+  UvwSParams<T> ap;
+  state_params(ap, P, gout, Y, phi, colptr, srcrecv, srcedge, S, N, E, P.c_out, NS, P.uvw_in, P.paths_adj, err);
+  for (int s0r = 0; s0r < N; s0r += NS) {
+    ap.r0 = s0r;
+    ap.nr = std::min(NS, N - s0r);
+    if ((e = build(ap, gout, dY, phi, 0, 1)) != cudaSuccess || (e = build(ap, gout, Y, dphi, 1, 1)) != cudaSuccess)
+      return cuda_fail(e, "uvw directional source state");
+    if ((e = mix_out<T>(P, S, pa.adj, pa.adj_lo, dgx, s0r, ap.nr, NS, P.uvw_in, ba_off, P.c_in, 0, err, s)) !=
+        cudaSuccess)
+      return cuda_fail(e, "uvw directional source mixing");
+    if ((e = build(ap, gout, Y, phi, 0, 1)) != cudaSuccess) return cuda_fail(e, "uvw source state");
+    if ((e = mix_out<T>(P, S, pd.adj, pd.adj_lo, dgx, s0r, ap.nr, NS, P.uvw_in, ba_off, P.c_in, 1, err, s)) !=
+        cudaSuccess)
+      return cuda_fail(e, "uvw source mixing");
+  }
+  e = launch_unpack_a<T>(P.pack, Ab, dgA, s);
+  return e == cudaSuccess ? TP_OK : cuda_fail(e, "unpack A_bar_dot");
 }
 
 }  // namespace
@@ -555,9 +715,14 @@ int tp_conv_launch_count(tp_plan_t plan, int64_t n_nodes, int pass, int* kernels
   const long long gin = ((long long)P.uvw_in.size() + kMaxGemmBatch - 1) / kMaxGemmBatch;
   if (pass == 0)
     *kernels = (int)(1 + cr * (1 + gout));                       // pack A; per chunk: state, mixing
-  else   // pack A; per receiver chunk: state, A_bar partials, their sum, S_bar, edge pass;
-         // per source chunk: source-view state, mixing; unpack A_bar
+  else if (pass == 1)   // pack A; per receiver chunk: state, A_bar partials, their sum, S_bar, edge pass;
+                        // per source chunk: source-view state, mixing; unpack A_bar
     *kernels = (int)(1 + cr * (1 + gout + 1 + gout + 1) + cs * (1 + gin) + 1);
+  else   // pack A and dA (twice each without tensor cores); per receiver chunk: three
+         // directional-state builds, mixing, A_bar_dot partials and their sum, the state,
+         // mixing, S_bar, two edge passes, dS_bar, one edge pass; per source chunk: three
+         // state builds, two mixings; unpack A_bar_dot
+    *kernels = (int)((P.uvw_tc ? 2 : 4) + cr * (8 + 5 * gout) + cs * (3 + 2 * gin) + 1);
   return TP_OK;
 }
 
@@ -681,8 +846,7 @@ int tp_conv_double_backward(tp_plan_t plan, const void* x, const void* Y, const 
     if (!al16(q)) return fail(TP_EINVAL, "floating-point buffers must be 16-byte aligned");
   if (n_edges > 0 && (!al16(Y) || !al16(phi) || !al16(dY) || !al16(dphi) || !al16(dgrad_Y) || !al16(dgrad_phi)))
     return fail(TP_EINVAL, "floating-point buffers must be 16-byte aligned");
-  if (P.mode == TP_UVW) return fail(TP_EUNSUPPORTED, "double backward of fully connected plans");
-  if (!P.dbl_ok) return fail(TP_EUNSUPPORTED, "double backward: more than 96 channel tiles of 32");
+  if (P.mode == TP_UVU && !P.dbl_ok) return fail(TP_EUNSUPPORTED, "double backward: more than 96 channel tiles of 32");
   const size_t need = workspace_bytes(P, n_nodes, 2);
   if (ws_bytes < need || (!ws && need > 0)) return fail(TP_EWORKSPACE, "workspace too small");
   int* err = nullptr;
@@ -696,6 +860,10 @@ int tp_conv_double_backward(tp_plan_t plan, const void* x, const void* Y, const 
   const int* idx[] = {rowptr, senders, colptr, srcedge, srcrecv};
   const void* dir[] = {dx, dY, dphi, dA};
   void* out[] = {d_out, dgrad_x, dgrad_Y, dgrad_phi, dgrad_A};
+  if (P.mode == TP_UVW)
+    return P.dtype == TP_F32
+               ? double_backward_uvw<float>(P, in, idx, dir, (int)n_nodes, (int)n_edges, out, ws, err, s)
+               : double_backward_uvw<double>(P, in, idx, dir, (int)n_nodes, (int)n_edges, out, ws, err, s);
   return P.dtype == TP_F32
              ? double_backward_uvu<float>(P, in, idx, dir, (int)n_nodes, (int)n_edges, out, ws, err, s)
              : double_backward_uvu<double>(P, in, idx, dir, (int)n_nodes, (int)n_edges, out, ws, err, s);

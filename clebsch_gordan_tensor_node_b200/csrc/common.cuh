@@ -128,6 +128,7 @@ struct UvwSParams {           // S (dir 0: receivers gather x) or S' (dir 1: sou
   T* S; int* err;
   int N, E, K, ld_feat, dim_y, n_feat_rows;
   int r0, nr, nr_alloc, n_blocks;
+  int accumulate;             // add to the state chunk instead of overwriting it
   UvwBlockD blocks[kMaxBlocks];
   PathD paths[kMaxPaths];     // x_off / mul_in describe the gathered block
 };
@@ -147,6 +148,7 @@ struct UvwEdgeParams {        // backward: edge-owned grad_phi, grad_Y from S_ba
   T* gY; T* gphi; int* err;
   int N, E, K, c_in, dim_y;
   int r0, nr, nr_alloc, n_blocks;
+  int accumulate;              // add to grad_phi / grad_Y instead of overwriting them
   int vec;                     // 16-byte copies: K == KP; c_in, x_off, mul_in multiples of 16 bytes
   int smem_stage, smem_sbar;   // bytes of one stage buffer (x part, then S_bar part) and its S_bar part
   int smem_red, smem_ct;       // bytes of the per-warp Y_bar region and of the C / T_bar columns

@@ -7,7 +7,7 @@
 // through one tiled kernel; the operands are addressed by small descriptors so
 // that output rows (receiver, component) land directly in the ir_mul output.
 //
-//   op NN:  C[m][n] = sum_k X[m][k] * B[k][n]      (m = S A, x_bar = S' A')
+//   op NN:  C[m][n] (+)= sum_k X[m][k] * B[k][n]   (m = S A, x_bar = S' A')
 //   op NT:  C[m][k] = sum_n G[m][n] * B[k][n]      (S_bar = m_bar A^T)
 //   op TN:  C[k][n] (+)= sum_m X[m][k] * G[m][n]   (A_bar += S^T m_bar)
 //
@@ -108,7 +108,8 @@ __global__ void __launch_bounds__(NT) gemm_kernel(const __grid_constant__ GemmBa
       const int gn = tn + tx * 2 + c;
       if (gn >= N) continue;
       if (OP == 0) {
-        blocked_row(p.C, p.c, gm)[gn] = acc[r][c];
+        T* dst = blocked_row(p.C, p.c, gm) + gn;
+        *dst = p.accumulate ? *dst + acc[r][c] : acc[r][c];
       } else if (OP == 1) {
         p.C[(size_t)gm * p.D + gn] = acc[r][c];
       } else {

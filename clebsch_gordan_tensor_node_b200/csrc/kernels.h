@@ -46,7 +46,7 @@ cudaError_t launch_pack_a(const UvwPackParams& p, const T* A, T* Bf, T* Ba, T* B
 template <typename T>
 cudaError_t launch_unpack_a(const UvwPackParams& p, const T* Bf, T* A, cudaStream_t s);
 
-// op 0: C = X B (C row-blocked); op 1: C = G B^T (dense); op 2: C (+)= X^T G (dense)
+// op 0: C (+)= X B (C row-blocked); op 1: C = G B^T (dense); op 2: C (+)= X^T G (dense)
 template <typename T>
 cudaError_t launch_gemm(int op, const GemmBatch<T>& gb, int n_prob, int max_m, int max_n, cudaStream_t s);
 // backward products: S_bar = m_bar B^T, and the split-K A_bar partials with
@@ -60,13 +60,13 @@ template <typename T>
 cudaError_t launch_sum_splits(const T* partial, size_t split_stride, int splits, T* out, long long n, int accumulate,
                               cudaStream_t s);
 
-// op 0 on tensor cores (fp32, 3xTF32): C = X Bt^T with X [M, D] and Bt [N, D]
+// op 0 on tensor cores (fp32, 3xTF32): C (+)= X Bt^T with X [M, D] and Bt [N, D]
 // row-major, read through TMA tensor maps (box 32 x 128 for X, 32 x N16 for Bt).
 struct TcProb {
   CUtensorMap tx, tbh, tbl;   // X (raw), Bt_hi, Bt_lo
   float* C;
   RowBlocked c;
-  int M, N, D, pad;
+  int M, N, D, accumulate;    // accumulate: add to C instead of overwriting it
 };
 struct TcBatch {
   TcProb prob[kMaxGemmBatch];

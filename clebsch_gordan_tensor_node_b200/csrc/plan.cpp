@@ -432,7 +432,11 @@ size_t workspace_bytes(const Plan& p, long long n_nodes, int pass) {
     const size_t s1 = ((size_t)uvw_chunk_rows(p, n_nodes, 1) * p.sa_row_elems * b + 255) / 256 * 256;
     // the tensor-core path adds the low parts of the transposed operands; the
     // backward adds the split-K partials of A_bar
-    const size_t na = pass == 0 ? (p.uvw_tc ? 2 : 1) : (p.uvw_tc ? 4 : 3) + kTnSplits;
+    // the double backward packs A and its direction for all three products
+    // (forward, source and S_bar operands; hi/lo on the tensor cores)
+    const size_t na = pass == 0   ? (p.uvw_tc ? 2 : 1)
+                      : pass == 1 ? (p.uvw_tc ? 4 : 3) + kTnSplits
+                                  : 2 * (p.uvw_tc ? 5 : 3) + 1 + kTnSplits;
     bytes = na * a + (pass == 0 ? s0 : 2 * std::max(s0, s1));
   }
   return (bytes + 255) / 256 * 256;

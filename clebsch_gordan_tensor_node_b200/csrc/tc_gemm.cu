@@ -252,14 +252,20 @@ __global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__
       if (row < M) {
         const int rb = row / p.c.dcomp, cc = row - rb * p.c.dcomp;
         float* dst = p.C + (size_t)(p.c.r0 + rb) * p.c.ld_outer + p.c.off + (size_t)cc * p.c.n;
+        if (p.accumulate) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (c0 + j < N) dst[c0 + j] = __uint_as_float(v[j]);
+          for (int j = 0; j < 32; ++j)
+            if (c0 + j < N) dst[c0 + j] += __uint_as_float(v[j]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c0 + j < N) dst[c0 + j] = __uint_as_float(v[j]);
+        }
       }
     }
   } else if (nkt == 0) {
     const int row = tm + warp * 32 + lane;
-    if (row < M) {
+    if (row < M && !p.accumulate) {
       const int rb = row / p.c.dcomp, cc = row - rb * p.c.dcomp;
       float* dst = p.C + (size_t)(p.c.r0 + rb) * p.c.ld_outer + p.c.off + (size_t)cc * p.c.n;
       for (int j = 0; j < N; ++j) dst[j] = 0.f;

@@ -181,8 +181,13 @@ __device__ __forceinline__ void sbuild_path(const UvwSParams<T>& p, const UvwBlo
           const int q = gid + 8 * h;
           if (q >= p.K) continue;
           T* row = dst + (size_t)m * bd.dcols + (size_t)q * gmul;
-          if (u < gmul) row[u] = acc[m][2 * h];
-          if (u + 1 < gmul) row[u + 1] = acc[m][2 * h + 1];
+          if (p.accumulate) {
+            if (u < gmul) row[u] += acc[m][2 * h];
+            if (u + 1 < gmul) row[u + 1] += acc[m][2 * h + 1];
+          } else {
+            if (u < gmul) row[u] = acc[m][2 * h];
+            if (u + 1 < gmul) row[u + 1] = acc[m][2 * h + 1];
+          }
         }
       }
     } else if (act) {
@@ -191,7 +196,10 @@ __device__ __forceinline__ void sbuild_path(const UvwSParams<T>& p, const UvwBlo
         const int qq = warp * KQ + q;
         if (qq < p.K) {
 #pragma unroll
-          for (int m = 0; m < DO; ++m) dst[(size_t)m * bd.dcols + (size_t)qq * gmul + cl] = Sr[q][m];
+          for (int m = 0; m < DO; ++m) {
+            T* o = dst + (size_t)m * bd.dcols + (size_t)qq * gmul + cl;
+            *o = p.accumulate ? *o + Sr[q][m] : Sr[q][m];
+          }
         }
       }
     }
@@ -484,12 +492,14 @@ uvw_edge_kernel(const __grid_constant__ UvwEdgeParams<T> p) {
         T acc = Rp[(size_t)v * 32 + sl];
 #pragma unroll
         for (int w = 1; w < kEdgeWarps; ++w) acc += Rp[((size_t)w * p.K + v) * 32 + sl];
+        if (p.accumulate) acc += p.gphi[eo * p.K + v];
         p.gphi[eo * p.K + v] = acc;
       } else {
         const int m = v - p.K;
         T acc = Red[(size_t)m * 32 + sl];
 #pragma unroll
         for (int w = 1; w < kEdgeWarps; ++w) acc += Red[((size_t)w * p.dim_y + m) * 32 + sl];
+        if (p.accumulate) acc += p.gY[eo * p.dim_y + m];
         p.gY[eo * p.dim_y + m] = acc;
       }
     }

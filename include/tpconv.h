@@ -223,8 +223,12 @@ int tp_conv_backward(tp_plan_t plan, const void* x, const void* Y, const void* p
  * edge order), dA [K, N_w]. Outputs (device, overwritten): d_out [N, C_out],
  * dgrad_x [N, C_in], dgrad_Y [E, dimY], dgrad_phi [E, K], dgrad_A [K, N_w].
  * ws: at least tp_conv_workspace_size(plan, N, 2) bytes. Results are bitwise
- * reproducible run to run (fixed ownership and order). Channelwise (uvu)
- * plans; TP_EUNSUPPORTED for fully connected plans. */
+ * reproducible run to run (fixed ownership and order). Fully connected (uvw)
+ * plans run the receiver program of Sobek §4.4 through the first-order
+ * kernels: the directional state dS = S(dx, Y, phi) + S(x, dY, phi) +
+ * S(x, Y, dphi) gives d_out = dS A + S dA and dgrad_A = dS^T grad_out; the
+ * edge pass runs on S_bar = grad_out A^T and dS_bar = grad_out dA^T; the
+ * source states give dgrad_x = (S'(dY, phi) + S'(Y, dphi)) A' + S' dA'. */
 int tp_conv_double_backward(tp_plan_t plan, const void* x, const void* Y, const void* phi, const void* A,
                             const int32_t* rowptr, const int32_t* senders, const int32_t* colptr,
                             const int32_t* srcedge, const int32_t* srcrecv, const void* grad_out,

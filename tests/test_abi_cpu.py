@@ -103,6 +103,10 @@ def test_launch_count_matches_the_schedule():
     # a graph small enough for one state chunk in each direction, one GEMM batch
     assert uvw.launch_count(100, 0) == 1 + 2
     assert uvw.launch_count(100, 1) == 1 + 5 + 2 + 1
+    # second order: pack A and dA; per receiver chunk 8 + 5 GEMM batches, per
+    # source chunk 3 + 2, unpack
+    assert uvw.launch_count(100, 2) == 2 + 13 + 5 + 1
+    assert uvu.launch_count(1000, 2) == 4
 
 
 def test_state_budget_sets_chunks_and_workspace():

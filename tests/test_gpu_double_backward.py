@@ -60,6 +60,31 @@ def test_double_backward_parity(cid, n):
         assert torch.equal(a, b)
 
 
+def test_double_backward_uvw_across_state_chunks():
+    """Fully connected workload at 200 nodes under a state budget of 60 nodes,
+    so the receiver program (directional state, mixings, three edge passes) and
+    the source states run over four chunks each."""
+    from test_gpu_parity import _state_row_bytes
+    cid = 5
+    wl = workload(cid, n_nodes=200)
+    plan = plan_for(cid)
+    s_row, sa_row = _state_row_bytes(plan)
+    plan.set_state_budget(60 * max(s_row, sa_row))
+    run = GpuRun(plan, wl)
+    d = _directions(wl, 12)
+    got = _dbl(run, d)
+    want = oconv.double_backward(problem(cid), wl.x, wl.Y, wl.phi, wl.A, wl.src, wl.dst, wl.grad_out, *d,
+                                 wl.n_nodes)
+    names = ("d_out", "dgrad_x", "dgrad_Y", "dgrad_phi", "dgrad_A")
+    for k, (g, w) in enumerate(zip(got, want)):
+        gn = run.to_coo(g) if k in (2, 3) else g.cpu().numpy()
+        assert rel_err(gn, w) <= TOL["f32"], names[k]
+    assert tpc.tp_get_device_error() == 0
+    again = _dbl(run, d)
+    for a, b in zip(got, again):
+        assert torch.equal(a, b)
+
+
 def test_double_backward_full_size_sampled():
     cid = 4
     wl = workload(cid)
