@@ -116,8 +116,8 @@ def setup(cid: int, dev: str, n_nodes=None):
     import clebsch_gordan_tensor_node_b200 as tpc
     from inputs import CONFIGS, make_workload
     c = CONFIGS[cid]
-    plan = tpc.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.K, c.mode, c.dtype)
-    wl = make_workload(cid, plan.n_w, n_nodes=n_nodes)
+    plan = tpc.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.K, c.mode, c.dtype, irreps_sh=c.irreps_sh)
+    wl = make_workload(cid, plan.n_w, n_nodes=n_nodes, c_out=plan.c_out)
     N, E = wl.n_nodes, wl.n_edges
     src = torch.from_numpy(wl.src.astype(np.int32)).to(dev)
     dst = torch.from_numpy(wl.dst.astype(np.int32)).to(dev)
@@ -289,8 +289,8 @@ class OracleSampler:
         self.oconv = oconv
         c = CONFIGS[cid]
         self.cid, self.both = cid, both and c.backward
-        self.pr = oconv.Problem(c.irreps_in, c.sh_lmax, c.irreps_out, c.K, c.mode)
-        self.wl = make_workload(cid, self.pr.n_w)
+        self.pr = oconv.Problem(c.irreps_in, c.sh_lmax, c.irreps_out, c.K, c.mode, c.irreps_sh)
+        self.wl = make_workload(cid, self.pr.n_w, c_out=self.pr.c_out)
         self.order = np.random.default_rng(0).permutation(self.wl.n_nodes)
         self.pos = 0
 

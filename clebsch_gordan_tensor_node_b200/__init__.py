@@ -10,7 +10,7 @@ from __future__ import annotations
 import ctypes
 from typing import Optional, Tuple
 
-from ._lib import (TP_F32, TP_F64, TP_UVU, TP_UVW, PathInfo, PlanInfo, TpConvError, check, lib)
+from ._lib import (TP_F32, TP_F64, TP_UVU, TP_UVU_PATHS, TP_UVW, PathInfo, PlanInfo, TpConvError, check, lib)
 
 __all__ = ["Plan", "tp_conv_plan", "tp_csr_build", "tp_csr_transpose", "tp_conv_forward",
            "tp_conv_backward", "tp_conv_double_backward", "tp_conv_backward_noalloc", "tp_get_device_error",
@@ -49,12 +49,16 @@ class Plan:
     """One convolution contract (tp_conv_plan). Host-only; owns no device memory."""
 
     def __init__(self, irreps_in: str, sh_lmax: int, irreps_out: str, n_radial: int,
-                 mode: str = "uvu", dtype: str = "f32"):
-        self.mode = {"uvu": TP_UVU, "uvw": TP_UVW}[mode]
+                 mode: str = "uvu", dtype: str = "f32", irreps_sh: Optional[str] = None):
+        self.mode = {"uvu": TP_UVU, "uvw": TP_UVW, "uvu_paths": TP_UVU_PATHS}[mode]
         self.dtype_code = {"f32": TP_F32, "f64": TP_F64}[dtype]
         h = ctypes.c_void_p()
-        check(lib().tp_conv_plan(irreps_in.encode(), sh_lmax, irreps_out.encode(), n_radial,
-                                 self.mode, self.dtype_code, ctypes.byref(h)), "tp_conv_plan")
+        if irreps_sh is None:
+            check(lib().tp_conv_plan(irreps_in.encode(), sh_lmax, irreps_out.encode(), n_radial,
+                                     self.mode, self.dtype_code, ctypes.byref(h)), "tp_conv_plan")
+        else:
+            check(lib().tp_conv_plan_sh(irreps_in.encode(), irreps_sh.encode(), irreps_out.encode(), n_radial,
+                                        self.mode, self.dtype_code, ctypes.byref(h)), "tp_conv_plan_sh")
         self._h = h
         info = PlanInfo()
         check(lib().tp_conv_plan_info(h, ctypes.byref(info)), "tp_conv_plan_info")

@@ -11,7 +11,7 @@ from ctypes import POINTER, c_char_p, c_double, c_int, c_int32, c_int64, c_size_
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtpconv.so")
 
-TP_UVU, TP_UVW = 0, 1
+TP_UVU, TP_UVW, TP_UVU_PATHS = 0, 1, 2
 TP_F32, TP_F64 = 0, 1
 STATUS = {0: "TP_OK", -1: "TP_EINVAL", -2: "TP_EUNSUPPORTED", -3: "TP_ECUDA",
           -4: "TP_EWORKSPACE", -5: "TP_EDEVICE_INDEX", -6: "TP_EDEVICE_CSR", -7: "TP_EDEVICE_TIMEOUT"}
@@ -33,6 +33,7 @@ class PathInfo(ctypes.Structure):
 # every exported symbol of tpconv.h with (restype, argtypes)
 SIGNATURES = {
     "tp_conv_plan": (c_int, [c_char_p, c_int, c_char_p, c_int, c_int, c_int, POINTER(c_void_p)]),
+    "tp_conv_plan_sh": (c_int, [c_char_p, c_char_p, c_char_p, c_int, c_int, c_int, POINTER(c_void_p)]),
     "tp_conv_plan_destroy": (c_int, [c_void_p]),
     "tp_conv_plan_info": (c_int, [c_void_p, POINTER(PlanInfo)]),
     "tp_conv_plan_path": (c_int, [c_void_p, c_int, POINTER(PathInfo)]),

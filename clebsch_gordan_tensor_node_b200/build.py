@@ -25,7 +25,7 @@ CG_LMAX = 6
 
 # translation units and how many instantiation sets each one is split into
 UNITS = {
-    "uvu_fwd.cu": 9,
+    "uvu_fwd.cu": 10,
     "uvu_bwd.cu": 10,
     "uvw.cu": 10,
     "uvu_dbwd.cu": 10,

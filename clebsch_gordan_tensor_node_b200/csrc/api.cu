@@ -74,8 +74,12 @@ cudaError_t fwd_prof(const Plan& P, const UvuFwdParams<T>& p, cudaStream_t s) {
     case 0: return launch_uvu_fwd<T, KP, CPL, 2, 2, 2>(p, s);
     case 1: return launch_uvu_fwd<T, KP, CPL, 1, 3, 3>(p, s);
     case 2: return launch_uvu_fwd<T, KP, CPL, 3, 3, 3>(p, s);
-    default:
+    case 3:
       if constexpr (Full) return launch_uvu_fwd<T, KP, CPL, 4, 4, 4>(p, s);
+      return cudaErrorInvalidValue;
+    default:   // degrees up to 6: fp32, K <= 8, one channel per lane
+      if constexpr (std::is_same<T, float>::value && KP == 8 && CPL == 1)
+        return launch_uvu_fwd<T, KP, CPL, 6, 6, 6>(p, s);
       return cudaErrorInvalidValue;
   }
 }
@@ -622,6 +626,27 @@ int tp_conv_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int
   return TP_OK;
 }
 
+int tp_conv_plan_sh(const char* irreps_in, const char* irreps_sh, const char* irreps_out, int n_radial, int mode,
+                    int dtype, tp_plan_t* plan) {
+  if (!plan) return fail(TP_EINVAL, "plan output pointer is NULL");
+  *plan = nullptr;
+  if (!irreps_sh) return fail(TP_EINVAL, "spherical-harmonic irreps string is NULL");
+  std::string msg;
+  int sh_lmax = 0;
+  std::vector<int> parity;
+  int st = parse_sh_irreps(irreps_sh, sh_lmax, parity, msg);
+  if (st != TP_OK) return fail(st, msg);
+  auto* h = new (std::nothrow) tp_plan_s;
+  if (!h) return fail(TP_EINVAL, "out of host memory");
+  st = make_plan(irreps_in, sh_lmax, irreps_out, n_radial, mode, dtype, h->p, msg, parity.data());
+  if (st != TP_OK) {
+    delete h;
+    return fail(st, msg);
+  }
+  *plan = h;
+  return TP_OK;
+}
+
 int tp_conv_plan_destroy(tp_plan_t plan) {
   delete plan;
   return TP_OK;
@@ -632,7 +657,7 @@ int tp_conv_plan_info(tp_plan_t plan, tp_plan_info_t* info) {
   const Plan& P = plan->p;
   std::memset(info, 0, sizeof(*info));
   info->c_in = P.c_in; info->c_out = P.c_out; info->dim_y = P.dim_y; info->n_radial = P.K;
-  info->n_paths = (int)P.paths.size(); info->mode = P.mode; info->dtype = P.dtype;
+  info->n_paths = (int)P.paths.size(); info->mode = P.per_path ? TP_UVU_PATHS : P.mode; info->dtype = P.dtype;
   info->sh_lmax = P.sh_lmax; info->lmax = P.lmax; info->n_w = P.n_w;
   return TP_OK;
 }

@@ -97,10 +97,11 @@ void add_tiles(const std::vector<Block>& blocks, const std::vector<std::vector<i
 }  // namespace
 
 int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_radial, int mode,
-              int dtype, Plan& P, std::string& msg) {
+              int dtype, Plan& P, std::string& msg, const int* sh_parity) {
   P = Plan{};
-  if (mode != TP_UVU && mode != TP_UVW) {
-    msg = "mode must be TP_UVU or TP_UVW";
+  auto par2 = [&](int l2) { return sh_parity ? sh_parity[l2] : ((l2 & 1) ? -1 : 1); };
+  if (mode != TP_UVU && mode != TP_UVW && mode != TP_UVU_PATHS) {
+    msg = "mode must be TP_UVU, TP_UVW or TP_UVU_PATHS";
     return TP_EINVAL;
   }
   if (dtype != TP_F32 && dtype != TP_F64) {
@@ -111,7 +112,35 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
     msg = "sh_lmax must be >= 0 and n_radial > 0";
     return TP_EINVAL;
   }
+  if (sh_lmax > 16) {
+    msg = "sh_lmax above 16";
+    return TP_EINVAL;
+  }
   if (!parse_irreps(irreps_in, P.bin, msg) || !parse_irreps(irreps_out, P.bout, msg)) return TP_EINVAL;
+  if (mode == TP_UVU_PATHS) {
+    // one output block per path (LunaTP Appendix A.1: per-path uvu outputs are
+    // concatenated): irreps_out only says which (l, p) exist; the output
+    // blocks are the paths' own, in enumeration order
+    std::vector<Block> allowed = P.bout;
+    P.bout.clear();
+    int off = 0;
+    for (const Block& b1 : P.bin)
+      for (int l2 = 0; l2 <= sh_lmax; ++l2)
+        for (int l3 = std::abs(b1.l - l2); l3 <= b1.l + l2; ++l3) {
+          const int p3 = b1.p * par2(l2);
+          bool ok = false;
+          for (const Block& a : allowed) ok |= (a.l == l3 && a.p == p3);
+          if (!ok) continue;
+          P.bout.push_back({b1.mul, l3, p3, off});
+          off += b1.mul * (2 * l3 + 1);
+        }
+    if (P.bout.empty()) {
+      msg = "no path reaches the output irreps";
+      return TP_EINVAL;
+    }
+    P.per_path = true;
+    mode = TP_UVU;
+  }
   P.mode = mode;
   P.dtype = dtype;
   P.K = n_radial;
@@ -123,10 +152,13 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
   for (size_t i1 = 0; i1 < P.bin.size(); ++i1) {
     const Block& b1 = P.bin[i1];
     for (int l2 = 0; l2 <= sh_lmax; ++l2) {
-      const int p2 = (l2 & 1) ? -1 : 1;
+      const int p2 = par2(l2);
       for (int l3 = std::abs(b1.l - l2); l3 <= b1.l + l2; ++l3) {
         const int p3 = b1.p * p2;
-        for (size_t io = 0; io < P.bout.size(); ++io) {
+        // per-path outputs: the path about to be added owns the next block
+        const size_t io0 = P.per_path ? P.paths.size() : 0;
+        const size_t io1 = P.per_path ? std::min(P.paths.size() + 1, P.bout.size()) : P.bout.size();
+        for (size_t io = io0; io < io1; ++io) {
           const Block& bo = P.bout[io];
           if (bo.l != l3 || bo.p != p3) continue;
           HostPath h{};
@@ -156,9 +188,12 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
   for (auto& b : P.bin) P.lmax = std::max(P.lmax, b.l);
   for (auto& b : P.bout) P.lmax = std::max(P.lmax, b.l);
   P.lmax = std::max(P.lmax, sh_lmax);
-  // limits of the compiled kernels
-  if (P.lmax > kLmax) {
-    msg = "degree " + std::to_string(P.lmax) + " above the kernels' limit " + std::to_string(kLmax);
+  // limits of the compiled kernels: degrees up to kLmax everywhere; up to
+  // kLmaxUvu for channelwise fp32 plans with K <= 8
+  const bool wide = mode == TP_UVU && dtype == TP_F32 && P.K <= 8;
+  if (P.lmax > (wide ? kLmaxUvu : kLmax)) {
+    msg = "degree " + std::to_string(P.lmax) + " above the kernels' limit " +
+          std::to_string(wide ? kLmaxUvu : kLmax) + " for this mode, dtype and K";
     return TP_EUNSUPPORTED;
   }
   if (P.K > 16) {
@@ -202,12 +237,14 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
   int lin = 0, lout = 0;
   for (auto& b : P.bin) lin = std::max(lin, b.l);
   for (auto& b : P.bout) lout = std::max(lout, b.l);
-  const int profs[4][3] = {{2, 2, 2}, {1, 3, 3}, {3, 3, 3}, {4, 4, 4}};
-  for (int k = 0; k < 4; ++k)
+  const int profs[5][3] = {{2, 2, 2}, {1, 3, 3}, {3, 3, 3}, {4, 4, 4}, {6, 6, 6}};
+  for (int k = 0; k < 5; ++k)
     if (lin <= profs[k][0] && sh_lmax <= profs[k][1] && lout <= profs[k][2]) {
       P.prof = k;
       break;
     }
+  // the widest profile is compiled for one channel per lane and scalar gathers
+  if (P.prof == 4) P.CPL = P.fwd_CPL = P.edge_V = 1;
   // instantiated combinations (uvu_fwd.cu): fp64 with 2 channels per lane only
   // with profiles 0-2
   if (dtype == TP_F64 && P.fwd_CPL == 2 && P.prof == 3) P.fwd_CPL = 1;
@@ -397,6 +434,21 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
       return TP_EUNSUPPORTED;
     }
   }
+  return TP_OK;
+}
+
+int parse_sh_irreps(const char* s, int& sh_lmax, std::vector<int>& parity, std::string& msg) {
+  std::vector<Block> b;
+  if (!parse_irreps(s, b, msg)) return TP_EINVAL;
+  parity.clear();
+  for (size_t k = 0; k < b.size(); ++k) {
+    if (b[k].l != (int)k || b[k].mul != 1) {
+      msg = "spherical-harmonic irreps must be 1x0?+1x1?+... with degrees 0, 1, 2, ... in order";
+      return TP_EINVAL;
+    }
+    parity.push_back(b[k].p);
+  }
+  sh_lmax = (int)b.size() - 1;
   return TP_OK;
 }
 

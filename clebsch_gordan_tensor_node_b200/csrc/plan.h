@@ -25,11 +25,12 @@ constexpr size_t kUvwChunkBytes = size_t(1) << 30;
 
 struct Plan {
   int mode = 0;     // 0 uvu, 1 uvw
+  bool per_path = false;    // uvu with one output block per path
   int dtype = 0;    // 0 f32, 1 f64
   int K = 0, KP = 0, CPL = 1, sh_lmax = 0, lmax = 0;
   int fwd_CPL = 1;          // channels per lane of the forward kernel
   int edge_V = 1;           // channels per gather in the uvu backward edge pass
-  int prof = 3;             // forward degree profile: 0 (2,2,2) 1 (1,3,3) 2 (3,3,3) 3 (4,4,4)
+  int prof = 3;             // degree profile: 0 (2,2,2) 1 (1,3,3) 2 (3,3,3) 3 (4,4,4) 4 (6,6,6)
   int cy_stride = 0, fwd_chunk = 32, fwd_warp_smem = 0;
   int fwd_ring_off = 0, fwd_ring_g = 1;   // forward: x copy ring offset (bytes); group size (= fwd_ring_g())
   int src_cy_stride = 0, src_chunk = 32, src_warp_smem = 0;
@@ -63,12 +64,18 @@ struct Plan {
 };
 
 
+// Parse spherical-harmonic irreps "1x0e+1x1o+..." (degrees 0..L in order,
+// multiplicity 1) into L and the parity of each degree.
+int parse_sh_irreps(const char* s, int& sh_lmax, std::vector<int>& parity, std::string& msg);
+
 // Owners per uvw state chunk for a problem of n_nodes nodes (dir 0: S, 1: S').
 int uvw_chunk_rows(const Plan& p, long long n_nodes, int dir);
 
 // Returns 0 or a negative tp_status; msg receives a human-readable reason.
+// sh_parity: parity (+1 / -1) of the spherical-harmonic block of each degree
+// 0..sh_lmax, or NULL for the natural parity (-1)^l.
 int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_radial, int mode,
-              int dtype, Plan& out, std::string& msg);
+              int dtype, Plan& out, std::string& msg, const int* sh_parity = nullptr);
 
 // Slots of the source pass's A_bar partial buffer (fixed per (plan, N)).
 int uvu_src_slots(const Plan& p, long long n_nodes);

@@ -3,9 +3,10 @@
 
 namespace tpc {
 
-constexpr int kLmax = 4;          // largest degree (l1, l2, l3) the kernels are built for
+constexpr int kLmax = 4;          // largest degree (l1, l2, l3) of the fully connected kernels
+constexpr int kLmaxUvu = 6;       // largest degree of the channelwise kernels (fp32, K <= 8 above kLmax)
 constexpr int kMaxPaths = 192;    // paths per plan (kernel parameter space)
-constexpr int kMaxTiles = 96;     // (block, channel tile) pairs per plan
+constexpr int kMaxTiles = 224;    // (block, channel tile) pairs per plan
 constexpr int kWarpsPerBlock = 8; // warps per CTA of the warp-task kernels
 constexpr int kSMs = 148;         // streaming multiprocessors of a B200
 constexpr int kTnSplits = 8;      // split-K partial copies of A_bar in the uvw backward

@@ -489,7 +489,11 @@ cudaError_t launch_uvu_edge(const UvuEdgeParams<T>& p0, int prof, cudaStream_t s
     case 0: return launch_edge_prof<T, KP, V, Prof<2, 2, 2>>(p, blocks, smem, s);
     case 1: return launch_edge_prof<T, KP, V, Prof<1, 3, 3>>(p, blocks, smem, s);
     case 2: return launch_edge_prof<T, KP, V, Prof<3, 3, 3>>(p, blocks, smem, s);
-    default: return launch_edge_prof<T, KP, V, Prof<4, 4, 4>>(p, blocks, smem, s);
+    case 3: return launch_edge_prof<T, KP, V, Prof<4, 4, 4>>(p, blocks, smem, s);
+    default:   // degrees up to 6: fp32, K <= 8, scalar gathers
+      if constexpr (std::is_same<T, float>::value && KP == 8 && V == 1)
+        return launch_edge_prof<T, KP, V, Prof<6, 6, 6>>(p, blocks, smem, s);
+      return cudaErrorInvalidValue;
   }
 }
 
@@ -514,7 +518,11 @@ cudaError_t launch_uvu_src(const UvuSrcParams<T>& p, int prof, cudaStream_t s) {
     case 0: return launch_src_prof<T, KP, CPL, Prof<2, 2, 2>>(p, blocks, s);
     case 1: return launch_src_prof<T, KP, CPL, Prof<1, 3, 3>>(p, blocks, s);
     case 2: return launch_src_prof<T, KP, CPL, Prof<3, 3, 3>>(p, blocks, s);
-    default: return launch_src_prof<T, KP, CPL, Prof<4, 4, 4>>(p, blocks, s);
+    case 3: return launch_src_prof<T, KP, CPL, Prof<4, 4, 4>>(p, blocks, s);
+    default:   // degrees up to 6: fp32, K <= 8, one channel per lane
+      if constexpr (std::is_same<T, float>::value && KP == 8 && CPL == 1)
+        return launch_src_prof<T, KP, CPL, Prof<6, 6, 6>>(p, blocks, s);
+      return cudaErrorInvalidValue;
   }
 }
 

@@ -423,15 +423,22 @@ __global__ void __launch_bounds__(kDbWarps * 32) uvu_dbwd_src_kernel(const __gri
   dispatch_l<PR::l1>(tl.l, [&](auto L) { src_tile<T, KP, PR, decltype(L)::value>(p, tl, slot, lane); });
 }
 
-template <typename F>
+// Wide: the degree-6 profile is compiled (fp32, K <= 8, scalar gathers only).
+template <bool Wide, typename F>
 cudaError_t by_prof(int prof, F&& f) {
   switch (prof) {
     case 0: return f(DProf<2, 2, 2>{});
     case 1: return f(DProf<1, 3, 3>{});
     case 2: return f(DProf<3, 3, 3>{});
-    default: return f(DProf<4, 4, 4>{});
+    case 3: return f(DProf<4, 4, 4>{});
+    default:
+      if constexpr (Wide) return f(DProf<6, 6, 6>{});
+      return cudaErrorInvalidValue;
   }
 }
+
+template <typename T, int KP>
+constexpr bool wide_ok() { return std::is_same<T, float>::value && KP == 8; }
 
 }  // namespace
 
@@ -440,7 +447,7 @@ cudaError_t launch_uvu_dbwd_recv(const UvuDbwdParams<T>& p, int prof, cudaStream
   const long long tasks = (long long)p.N * p.n_tiles;
   if (tasks == 0) return cudaSuccess;
   const unsigned blocks = (unsigned)((tasks + kDbWarps - 1) / kDbWarps);
-  return by_prof(prof, [&](auto PR) {
+  return by_prof<wide_ok<T, KP>()>(prof, [&](auto PR) {
     uvu_dbwd_recv_kernel<T, KP, decltype(PR)><<<blocks, kDbWarps * 32, 0, s>>>(p);
     return cudaGetLastError();
   });
@@ -454,7 +461,7 @@ cudaError_t launch_uvu_dbwd_edge(const UvuDbwdParams<T>& p0, int prof, cudaStrea
   p.split = groups < kDbSplitGroups ? kDbWarps : 1;
   const unsigned blocks = (unsigned)(p.split > 1 ? groups : (groups + kDbWarps - 1) / kDbWarps);
   const size_t smem = p.split > 1 ? sizeof(T) * (size_t)kDbWarps * (p.K + p.dim_y) * 32 : 0;
-  return by_prof(prof, [&](auto PR) {
+  return by_prof<wide_ok<T, KP>() && V == 1>(prof, [&](auto PR) {
     auto kern = uvu_dbwd_edge_kernel<T, KP, V, decltype(PR)>;
     static SmemLimit limit;
     if (cudaError_t e = limit.ensure((const void*)kern, smem); e != cudaSuccess) return e;
@@ -469,7 +476,7 @@ cudaError_t launch_uvu_dbwd_src(const UvuDbwdParams<T>& p, int prof, cudaStream_
   if (err != cudaSuccess) return err;
   if (p.n_slots == 0 || p.n_tiles == 0 || p.N == 0) return cudaSuccess;
   const unsigned blocks = (unsigned)(((long long)p.n_slots + kDbWarps - 1) / kDbWarps * p.n_tiles);
-  return by_prof(prof, [&](auto PR) {
+  return by_prof<wide_ok<T, KP>()>(prof, [&](auto PR) {
     uvu_dbwd_src_kernel<T, KP, decltype(PR)><<<blocks, kDbWarps * 32, 0, s>>>(p);
     return cudaGetLastError();
   });

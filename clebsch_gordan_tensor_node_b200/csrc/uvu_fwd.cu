@@ -294,6 +294,9 @@ TPC_INST(float, 8, 1, 4, 4, 4)
 #if TPC_WANT(1)
 TPC_INST_P(float, 8, 2)
 #endif
+#if TPC_WANT(9)
+TPC_INST(float, 8, 1, 6, 6, 6)
+#endif
 #if TPC_WANT(2)
 TPC_INST(float, 8, 2, 4, 4, 4)
 #endif

@@ -60,7 +60,7 @@ extern "C" {
 
 typedef struct tp_plan_s* tp_plan_t;
 
-enum tp_mode { TP_UVU = 0, TP_UVW = 1 };
+enum tp_mode { TP_UVU = 0, TP_UVW = 1, TP_UVU_PATHS = 2 };
 enum tp_dtype { TP_F32 = 0, TP_F64 = 1 };
 enum tp_status {
   TP_OK = 0,
@@ -97,16 +97,34 @@ typedef struct {
 /* Plan one convolution contract (Sobek §4.5: validate the contract, enumerate
  * the valid paths and their sparse CG terms; §2.2 for the selection rule).
  * irreps_in / irreps_out: strings such as "64x0e+64x1o+64x2e". sh_lmax: degree
- * of Y. n_radial: K. mode: TP_UVU or TP_UVW. dtype: TP_F32 or TP_F64.
- * Paths are enumerated for each input block in order, l2 = 0..sh_lmax
+ * of Y. n_radial: K. mode: TP_UVU, TP_UVW or TP_UVU_PATHS. dtype: TP_F32 or
+ * TP_F64. Paths are enumerated for each input block in order, l2 = 0..sh_lmax
  * ascending (Y of parity (-1)^l2), l3 = |l1-l2|..l1+l2 ascending, one path per
  * output block of that degree and parity; output blocks sum their paths.
+ * TP_UVU_PATHS is the channelwise product with one output block per path
+ * (LunaTP Appendix A.1: the uvu paths' outputs are concatenated): irreps_out
+ * only says which (l, p) may be produced (its multiplicities are ignored); the
+ * output row holds, in path order, one block of the path's input multiplicity
+ * and degree l3 per path (tp_conv_plan_info gives C_out, tp_conv_plan_path the
+ * blocks' offsets). Degrees up to 4 are compiled for every mode and dtype, up
+ * to 6 for channelwise fp32 plans with K <= 8.
  * Host only (no CUDA call). On success *plan receives a new plan that the
  * caller releases with tp_conv_plan_destroy. Errors: TP_EINVAL (malformed
- * string, bad enum, NULL), TP_EUNSUPPORTED (uvu with unequal multiplicity on a
- * path, degree above 4, K above 16, too many paths). */
+ * string, bad enum, NULL, no path reaches the outputs), TP_EUNSUPPORTED (uvu
+ * with unequal multiplicity on a path, degree above the limit, K above 16,
+ * more than 192 paths or 224 channel tiles). */
 int tp_conv_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_radial,
                  int mode, int dtype, tp_plan_t* plan);
+
+/* tp_conv_plan with the spherical-harmonic irreps given explicitly, as
+ * "1x0e+1x1o+1x2e" (degrees 0..L in order, multiplicity 1): the parity of
+ * each degree of Y is taken from the string instead of (-1)^l. Parity only
+ * selects the paths (Sobek §2.2: p_out = p_in p_sh); the arithmetic of Y is
+ * unchanged. Used by contracts whose edge irreps are all even (LunaTP
+ * Appendix A.1, Table 1, case C1). Errors as tp_conv_plan, plus TP_EINVAL for a
+ * malformed SH string. */
+int tp_conv_plan_sh(const char* irreps_in, const char* irreps_sh, const char* irreps_out, int n_radial,
+                    int mode, int dtype, tp_plan_t* plan);
 
 /* Release a plan (NULL is accepted). */
 int tp_conv_plan_destroy(tp_plan_t plan);

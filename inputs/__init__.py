@@ -5,4 +5,4 @@ features, weights, output cotangents). It holds none of the convolution's
 arithmetic, imports neither the CUDA path nor the oracle, and is the one module
 both sides see.
 """
-from .workloads import CONFIGS, Workload, make_workload  # noqa: F401
+from .workloads import CONFIGS, LUNATP_CASES, Workload, make_workload  # noqa: F401

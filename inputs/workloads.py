@@ -47,6 +47,7 @@ class Config:
     a_std: float
     backward: bool
     positions_from: int = 0   # reuse another workload's positions
+    irreps_sh: Optional[str] = None   # parities of Y's degrees where not (-1)^l
 
 
 def _lp(mul: int, lmax: int, all_parities: bool, skip=()) -> str:
@@ -81,6 +82,39 @@ CONFIGS = {
               "32x0e+32x1o+32x2e+32x3o+32x4e", 4, _lp(32, 4, True), 16, "uvw", "f32",
               16_384, _box(16_384, 32.0, 5.0), True, 5.0, 1.0 / np.sqrt(16.0 * 32.0), True),
 }
+
+
+# The ten irrep cases of LunaTP's kernel microbenchmarks (Appendix A.1, Table 1:
+# hidden, edge and output irreps), on their workload's shape: 768 atoms,
+# periodic, r_c 6 A, 48.6 neighbours on average (OMat24 structures there;
+# uniform positions here). Outputs are per path (mode "uvu_paths"): the output
+# irreps listed select which (l, p) the paths may produce. K = 8 Bessel
+# functions give the per-edge path weights through W = phi A.
+_LUNATP = [
+    ("C1", "128x0e+64x1e+32x2e", "1x0e+1x1e+1x2e", "224x0e+384x1e+352x2e"),
+    ("C2", "128x0e+128x1o+128x2e", "1x0e+1x1o+1x2e+1x3o", "384x0e+640x1o+640x2e+512x3o"),
+    ("C3", "128x0e+64x1o+32x2e+32x3o", "1x0e+1x1o+1x2e+1x3o", "256x0e+352x1o+384x2e+320x3o"),
+    ("C4", "256x0e+256x1o+256x2e+256x3o", "1x0e+1x1o+1x2e+1x3o", "1024x0e+1536x1o+1792x2e+1536x3o"),
+    ("C5", "320x0e+96x1o+64x2e+32x3o+32x4e", "1x0e+1x1o+1x2e+1x3o+1x4e",
+     "544x0e+736x1o+832x2e+800x3o+704x4e"),
+    ("C6", "128x0e+128x1o+128x2e+128x3o+128x4e", "1x0e+1x1o+1x2e+1x3o+1x4e",
+     "640x0e+1024x1o+1280x2e+1280x3o+1152x4e"),
+    ("C7", "128x0e+64x1o+32x2e+32x3o+32x4e+32x5o", "1x0e+1x1o+1x2e+1x3o+1x4e+1x5o",
+     "320x0e+480x1o+576x2e+608x3o+608x4e+512x5o"),
+    ("C8", "96x0e+96x1o+96x2e+96x3o+96x4e+96x5o", "1x0e+1x1o+1x2e+1x3o+1x4e+1x5o",
+     "576x0e+960x1o+1248x2e+1344x3o+1344x4e+1152x5o"),
+    ("C9", "128x0e+64x1o+32x2e+32x3o+32x4e+32x5o+32x6e", "1x0e+1x1o+1x2e+1x3o+1x4e+1x5o+1x6e",
+     "352x0e+544x1o+672x2e+736x3o+768x4e+736x5o+640x6e"),
+    ("C10", "64x0e+64x1o+64x2e+64x3o+64x4e+64x5o+64x6e", "1x0e+1x1o+1x2e+1x3o+1x4e+1x5o+1x6e",
+     "448x0e+768x1o+1024x2e+1152x3o+1216x4e+1152x5o+1024x6e"),
+]
+for _k, (_name, _hid, _sh, _out) in enumerate(_LUNATP):
+    _cid = 11 + _k
+    _lsh = len(_sh.split("+")) - 1
+    CONFIGS[_cid] = Config(_cid, f"LunaTP {_name} f32 per-path uvu (768 atoms, ~48.6 nbrs, r_c 6 A, L_sh {_lsh})",
+                           _hid, _lsh, _out, 8, "uvu_paths", "f32", 768, _box(768, 48.6, 6.0), True, 6.0,
+                           1.0 / np.sqrt(8.0), True, irreps_sh=_sh)
+LUNATP_CASES = {name: 11 + k for k, (name, *_r) in enumerate(_LUNATP)}
 
 
 def _positions(cfg: Config, rng: np.random.Generator) -> np.ndarray:
@@ -174,10 +208,11 @@ class Workload:
 
 
 def make_workload(cfg_id: int, n_w: int, n_nodes: Optional[int] = None,
-                  edge_keep: Optional[float] = None) -> Workload:
+                  edge_keep: Optional[float] = None, c_out: Optional[int] = None) -> Workload:
     """Build workload ``cfg_id``.
 
-    n_w (the weight count of the operator's path layout) is an argument so that
+    n_w (the weight count of the operator's path layout) and c_out (the output
+    width, needed where the paths define the output blocks) are arguments so that
     this module stays free of the operator's path rules. ``n_nodes`` shrinks a
     periodic workload at fixed density (for fast tests); ``edge_keep`` keeps a
     seeded fraction of the edges (for workspace-versus-edge-count checks).
@@ -205,5 +240,5 @@ def make_workload(cfg_id: int, n_w: int, n_nodes: Optional[int] = None,
     phi = bessel_cutoff(r, cfg.K, cfg.r_cut).astype(dt)
     x = rng.normal(size=(cfg.n_nodes, _irreps_dim(cfg.irreps_in))).astype(dt)
     A = (rng.normal(size=(cfg.K, n_w)) * cfg.a_std).astype(dt)
-    g = rng.normal(size=(cfg.n_nodes, _irreps_dim(cfg.irreps_out))).astype(dt)
+    g = rng.normal(size=(cfg.n_nodes, c_out if c_out is not None else _irreps_dim(cfg.irreps_out))).astype(dt)
     return Workload(cfg, pos, src, dst, Y, phi, x, A, g, n_w)

@@ -27,13 +27,13 @@ in any order; all arithmetic is fp64.
 from __future__ import annotations
 
 from dataclasses import dataclass
-from typing import List
+from typing import List, Optional
 
 import numpy as np
 
 from . import irreps as _ir
 from .cg import real_cg
-from .paths import Path, enumerate_paths, n_weights, y_offset
+from .paths import Path, enumerate_paths, n_weights, per_path_irreps_out, y_offset
 
 
 @dataclass
@@ -43,12 +43,21 @@ class Problem:
     irreps_out: str
     K: int
     mode: str
+    irreps_sh: Optional[str] = None   # explicit parities of Y's degrees ("1x0e+1x1e+...")
 
     def __post_init__(self):
         self.bin = _ir.parse(self.irreps_in)
+        sh = self.sh_lmax
+        if self.irreps_sh is not None:
+            sh = [(b.l, b.p) for b in _ir.parse(self.irreps_sh)]
+            assert [l for l, _ in sh] == list(range(self.sh_lmax + 1))
+        self.paths: List[Path] = enumerate_paths(self.irreps_in, sh, self.irreps_out, self.mode)
+        if self.mode == "uvu_paths":
+            # one output block per path (LunaTP Appendix A.1): irreps_out only
+            # selects which (l, p) exist; each path is channelwise on its block
+            self.irreps_out = per_path_irreps_out(self.irreps_in, sh, self.irreps_out)
+            self.mode = "uvu"
         self.bout = _ir.parse(self.irreps_out)
-        self.paths: List[Path] = enumerate_paths(self.irreps_in, self.sh_lmax,
-                                                 self.irreps_out, self.mode)
         self.c_in = _ir.dim(self.bin)
         self.c_out = _ir.dim(self.bout)
         self.dim_y = (self.sh_lmax + 1) ** 2
@@ -69,8 +78,9 @@ def _blocks(pr: Problem, p: Path, x, Y, src):
 
 
 def _chunk(pr: Problem, chunk: int) -> int:
-    """Edges per materialised chunk, bounded so that W [chunk, N_w] stays <= 1 GiB."""
-    return max(1, min(chunk, (1 << 27) // max(1, pr.n_w)))
+    """Edges per materialised chunk, bounded so that W [chunk, N_w] and the edge
+    messages [chunk, C_out] (and their adjoints) each stay <= 1 GiB."""
+    return max(1, min(chunk, (1 << 27) // max(1, pr.n_w, pr.c_out, pr.c_in)))
 
 
 def forward(pr: Problem, x, Y, phi, A, src, dst, n_nodes: int, chunk: int = 65536):

@@ -50,7 +50,45 @@ def y_offset(l2: int) -> int:
     return l2 * l2
 
 
+def per_path_irreps_out(irreps_in: str, sh, irreps_out: str) -> str:
+    """Output irreps of the channelwise convolution with one output block per path
+    (LunaTP Appendix A.1, Table 1: the outputs of the uvu paths are concatenated).
+
+    Paths are enumerated in the same order as ``enumerate_paths``; a path exists
+    when its (l3, p3) appears in ``irreps_out`` (multiplicities there are
+    ignored), and it owns a block of its input multiplicity.
+    """
+    bin_ = _ir.parse(irreps_in)
+    allowed = {(b.l, b.p) for b in _ir.parse(irreps_out)}
+    terms = []
+    for b1 in bin_:
+        for (l2, p2) in sh_irreps(sh):
+            for l3 in range(abs(b1.l - l2), b1.l + l2 + 1):
+                p3 = b1.p * p2
+                if (l3, p3) in allowed:
+                    terms.append(f"{b1.mul}x{l3}{'e' if p3 == 1 else 'o'}")
+    return "+".join(terms)
+
+
 def enumerate_paths(irreps_in: str, sh, irreps_out: str, mode: str) -> List[Path]:
+    """Paths in enumeration order. mode "uvu" / "uvw": every output block of the
+    right (l3, p3) receives a path and sums its paths; mode "uvu_paths": one
+    output block per path, in path order (``irreps_out`` only selects which
+    (l3, p3) exist; the blocks are those of ``per_path_irreps_out``)."""
+    if mode == "uvu_paths":
+        bin_ = _ir.parse(irreps_in)
+        allowed = {(b.l, b.p) for b in _ir.parse(irreps_out)}
+        paths = []
+        w = 0
+        for i1, b1 in enumerate(bin_):
+            for (l2, p2) in sh_irreps(sh):
+                for l3 in range(abs(b1.l - l2), b1.l + l2 + 1):
+                    p3 = b1.p * p2
+                    if (l3, p3) in allowed:
+                        k = len(paths)
+                        paths.append(Path(k, i1, b1.l, b1.p, l2, p2, l3, p3, k, b1.mul, b1.mul, w, b1.mul))
+                        w += b1.mul
+        return paths
     bin_ = _ir.parse(irreps_in)
     bout = _ir.parse(irreps_out)
     shl = sh_irreps(sh)
@@ -136,7 +174,7 @@ def work_model(paths: List[Path], n_nodes: int, n_edges: int, K: int, mode: str)
         nnz = len(real_cg_sparse(p.l1, p.l2, p.l3))
         d1 = 2 * p.l1 + 1
         d3 = 2 * p.l3 + 1
-        if mode == "uvu":
+        if mode in ("uvu", "uvu_paths"):
             C = p.mul_in
             fwd += 2 * n_edges * C * (K + nnz + d3)
             bwd += 2 * n_edges * C * (3 * K + 3 * nnz + 2 * d3)

@@ -23,16 +23,17 @@ def rel_err(got, want) -> float:
 
 def problem(cid: int) -> Problem:
     c = CONFIGS[cid]
-    return Problem(c.irreps_in, c.sh_lmax, c.irreps_out, c.K, c.mode)
+    return Problem(c.irreps_in, c.sh_lmax, c.irreps_out, c.K, c.mode, c.irreps_sh)
 
 
 def plan_for(cid: int) -> tpc.Plan:
     c = CONFIGS[cid]
-    return tpc.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.K, c.mode, c.dtype)
+    return tpc.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.K, c.mode, c.dtype, irreps_sh=c.irreps_sh)
 
 
 def workload(cid: int, n_nodes=None, edge_keep=None):
-    return make_workload(cid, problem(cid).n_w, n_nodes=n_nodes, edge_keep=edge_keep)
+    pr = problem(cid)
+    return make_workload(cid, pr.n_w, n_nodes=n_nodes, edge_keep=edge_keep, c_out=pr.c_out)
 
 
 class GpuRun:

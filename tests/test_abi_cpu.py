@@ -17,6 +17,13 @@ from oracle import paths as opaths
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
+def _sh(c):
+    """Y's degrees and parities of a workload (natural parity unless given)."""
+    if c.irreps_sh is None:
+        return c.sh_lmax
+    return [(int(t.split("x")[1][:-1]), 1 if t[-1] == "e" else -1) for t in c.irreps_sh.split("+")]
+
+
 def _declared():
     txt = open(os.path.join(ROOT, "include", "tpconv.h")).read()
     return sorted(set(re.findall(r"^\s*(?:int|const char\*)\s+(tp_\w+)\s*\(", txt, re.M)))
@@ -34,8 +41,8 @@ def test_library_exports_every_declared_symbol():
 @pytest.mark.parametrize("cid", sorted(CONFIGS))
 def test_planner_matches_oracle_paths(cid):
     c = CONFIGS[cid]
-    plan = tpc.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.K, c.mode, c.dtype)
-    ps = opaths.enumerate_paths(c.irreps_in, c.sh_lmax, c.irreps_out, c.mode)
+    plan = tpc.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.K, c.mode, c.dtype, irreps_sh=c.irreps_sh)
+    ps = opaths.enumerate_paths(c.irreps_in, _sh(c), c.irreps_out, c.mode)
     assert plan.n_paths == len(ps)
     assert plan.n_w == opaths.n_weights(ps)
     for k, p in enumerate(ps):
@@ -60,8 +67,8 @@ def test_planner_cg_matches_oracle():
 @pytest.mark.parametrize("cid", sorted(CONFIGS))
 def test_work_model_matches_oracle(cid):
     c = CONFIGS[cid]
-    plan = tpc.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.K, c.mode, c.dtype)
-    ps = opaths.enumerate_paths(c.irreps_in, c.sh_lmax, c.irreps_out, c.mode)
+    plan = tpc.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.K, c.mode, c.dtype, irreps_sh=c.irreps_sh)
+    ps = opaths.enumerate_paths(c.irreps_in, _sh(c), c.irreps_out, c.mode)
     N, E = 1000, 31000
     want = opaths.work_model(ps, N, E, c.K, c.mode)
     assert plan.work_model(N, E, 0)[0] == pytest.approx(want["fwd_flops"], rel=1e-12)
@@ -83,7 +90,11 @@ def test_workspace_does_not_depend_on_edges():
     (("8x0e+", 1, "8x0e", 8, "uvu", "f32"), -1),
     (("8x0e", 1, "8x0q", 8, "uvu", "f32"), -1),
     (("8x0e", 1, "4x1o", 8, "uvu", "f32"), -2),     # uvu with unequal multiplicity
-    (("8x5e", 1, "8x5e", 8, "uvu", "f32"), -2),     # degree above the compiled limit
+    (("8x7e", 1, "8x7e", 8, "uvu", "f32"), -2),     # degree above the compiled limit (6)
+    (("8x5e", 1, "8x5e", 8, "uvw", "f32"), -2),     # fully connected: limit 4
+    (("8x5e", 1, "8x5e", 8, "uvu", "f64"), -2),     # fp64: limit 4
+    (("8x5e", 1, "8x5e", 16, "uvu", "f32"), -2),    # K above 8: limit 4
+    (("8x0e", 1, "8x3o", 8, "uvu_paths", "f32"), -1),   # no path reaches the outputs
     (("8x0e", 1, "8x0e", 33, "uvu", "f32"), -2),    # K above 16
 ])
 def test_plan_errors(args, status):
@@ -126,3 +137,31 @@ def test_state_budget_sets_chunks_and_workspace():
     uvu = tpc.Plan("8x0e", 0, "8x0e", 4, "uvu", "f32")
     uvu.set_state_budget(1)            # no state chunks: accepted, no effect
     assert uvu.workspace_size(10, 0) == 0
+
+
+def test_per_path_outputs_match_lunatp_table1():
+    """Per-path (concatenated) channelwise outputs: the planner's output blocks,
+    summed per (l, p), give the output multiplicities of LunaTP Appendix A.1,
+    Table 1 for all ten cases, and every block belongs to exactly one path."""
+    from inputs import LUNATP_CASES
+    gold = {}
+    for line in open(os.path.join(ROOT, "tests", "golden", "lunatp_table1_out_mul.txt")):
+        if line.strip() and not line.startswith("#"):
+            case, _, _, out = [c.strip() for c in line.split("|")]
+            gold[case] = {}
+            for t in out.split("+"):
+                mul, ir = t.split("x")
+                gold[case][(int(ir[:-1]), 1 if ir[-1] == "e" else -1)] = int(mul)
+    for case, cid in LUNATP_CASES.items():
+        c = CONFIGS[cid]
+        plan = tpc.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.K, c.mode, c.dtype, irreps_sh=c.irreps_sh)
+        assert plan.info.mode == 2
+        tot = {}
+        outs = set()
+        for k in range(plan.n_paths):
+            p = plan.path(k)
+            assert p.block_out == k and p.mul_out == p.mul_in
+            outs.add(p.out_off)
+            tot[(p.l3, p.p3)] = tot.get((p.l3, p.p3), 0) + p.mul_in
+        assert tot == gold[case], case
+        assert len(outs) == plan.n_paths
