@@ -593,6 +593,131 @@ def workspace_vs_edges(dev, head):
     return rec
 
 
+# ----------------------------------------------------------------------------- scaling sweeps
+
+# Sobek §5.1: fully connected profiles, in = out irreps with alternating
+# parity, one SH copy per order, K = 16, 128 MiB receiver scratch budget.
+SWEEP_PROFILES = ("128/64", "128/64/64", "128/64/64/64")
+# Sobek Table 3: the sixteen capacity-matched profiles with OpenEquivariance's
+# largest graph counts for forward, backward and double backward (copies of the
+# 128-node, degree-32 graph).
+TABLE3 = (("32/16", 862, 431, 215), ("32/32", 487, 243, 121), ("32/16/16", 433, 216, 108),
+          ("32/32/32", 178, 88, 44), ("32/16/16/16", 244, 121, 60), ("32/32/32/32", 85, 42, 21),
+          ("64/32", 217, 108, 54), ("64/64", 122, 61, 30), ("64/32/32", 108, 54, 27),
+          ("64/64/64", 44, 22, 11), ("64/32/32/32", 61, 30, 15), ("64/64/64/64", 21, 10, 5),
+          ("128/64", 54, 27, 13), ("128/128", 30, 15, 7), ("128/64/64", 27, 13, 6), ("128/64/64/64", 15, 7, 3))
+
+
+def profile_irreps(profile: str):
+    muls = [int(v) for v in profile.split("/")]
+    return "+".join(f"{m}x{l}{'e' if l % 2 == 0 else 'o'}" for l, m in enumerate(muls)), len(muls) - 1
+
+
+def _sweep_point(plan, graph, dev, passes, budget_s=0.25):
+    """Median CUDA-event time (ms) and peak allocated memory of each pass on one
+    graph: at least 5 warm-up calls and 50 ms, then 10-30 samples totalling at
+    least `budget_s` (fewer for calls above a second)."""
+    import torch
+
+    import clebsch_gordan_tensor_node_b200 as tpc
+    from inputs import sobek_workload
+    irreps = plan.irreps
+    w = sobek_workload(graph, irreps, plan.sh_lmax, plan.n_radial, plan.n_w, plan.c_out)
+    N, E = w["n_nodes"], len(w["src"])
+    src = torch.from_numpy(w["src"].astype(np.int32)).to(dev)
+    dst = torch.from_numpy(w["dst"].astype(np.int32)).to(dev)
+    rowptr, senders, perm = tpc.tp_csr_build(src, dst, N)
+    colptr, srcedge, srcrecv = tpc.tp_csr_transpose(rowptr, senders, N)
+    p = perm.long()
+    x = torch.from_numpy(w["x"]).to(dev)
+    Y = torch.from_numpy(w["Y"]).to(dev)[p].contiguous()
+    phi = torch.from_numpy(w["phi"]).to(dev)[p].contiguous()
+    A = torch.from_numpy(w["A"]).to(dev)
+    g = torch.from_numpy(w["grad_out"]).to(dev)
+    del src, dst, p
+    calls = {
+        "fwd": lambda: tpc.tp_conv_forward(plan, x, Y, phi, A, rowptr, senders),
+        "bwd": lambda: tpc.tp_conv_backward(plan, x, Y, phi, A, rowptr, senders, colptr, srcedge, srcrecv, g),
+        "dbl": lambda: tpc.tp_conv_double_backward(plan, x, Y, phi, A, rowptr, senders, colptr, srcedge, srcrecv,
+                                                   g, x, Y, phi, A),
+    }
+    out = {"nodes": N, "edges": E}
+    for name in passes:
+        f = calls[name]
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        n = 0
+        while n < 5 or time.perf_counter() - t0 < 0.05:
+            f()
+            torch.cuda.synchronize()
+            n += 1
+            if time.perf_counter() - t0 > 3.0 and n >= 2:
+                break
+        torch.cuda.reset_peak_memory_stats()
+        times = []
+        while len(times) < 30:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            f()
+            b.record()
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+            if (len(times) >= 10 and sum(times) >= budget_s * 1e3) or (len(times) >= 3 and sum(times) > 3e3):
+                break
+        ms = statistics.median(times)
+        out[name] = {"ms": round(ms, 4), "M_edges_per_s": round(E / (ms * 1e-3) / 1e6, 2),
+                     "peak_GiB": round(torch.cuda.max_memory_allocated() / 2 ** 30, 3), "samples": len(times)}
+    assert tpc.tp_get_device_error() == 0
+    return out
+
+
+def _sweep_plan(profile):
+    import clebsch_gordan_tensor_node_b200 as tpc
+    irreps, L = profile_irreps(profile)
+    plan = tpc.Plan(irreps, L, irreps, 16, "uvw", "f32")
+    plan.irreps, plan.sh_lmax = irreps, L
+    try:
+        plan.set_state_budget(128 << 20)
+    except tpc.TpConvError:
+        pass   # one node's state is larger: keep the default budget
+    return plan
+
+
+def run_sweeps(args):
+    """Sobek §5.1-5.4 workloads: degree and graph-count scaling of the three
+    scaling profiles, and the capacity-matched sixteen-profile grid of Table 3.
+    Prints one JSON line."""
+    import torch
+
+    from inputs import SOBEK_COUNTS, SOBEK_DEGREES, sobek_count_graph, sobek_degree_graph
+    dev = "cuda:0"
+    torch.cuda.set_device(dev)
+    res = {"kind": "sobek sweeps", "state_budget_bytes": 128 << 20, "K": 16, "dtype": "f32",
+           "degree": {}, "graph_count": {}, "table3": []}
+    passes = ("fwd", "bwd", "dbl")
+    if "degree" in args.sweeps:
+        for prof in SWEEP_PROFILES:
+            plan = _sweep_plan(prof)
+            res["degree"][prof] = [dict(degree=d, **_sweep_point(plan, sobek_degree_graph(d), dev, passes))
+                                   for d in SOBEK_DEGREES]
+            torch.cuda.empty_cache()
+    if "count" in args.sweeps:
+        for prof in SWEEP_PROFILES:
+            plan = _sweep_plan(prof)
+            res["graph_count"][prof] = [dict(copies=b, **_sweep_point(plan, sobek_count_graph(b), dev, passes))
+                                        for b in SOBEK_COUNTS]
+            torch.cuda.empty_cache()
+    if "table3" in args.sweeps:
+        for prof, bf, bb, bd in TABLE3:
+            plan = _sweep_plan(prof)
+            row = {"profile": prof, "n_w": plan.n_w}
+            for name, b in (("fwd", bf), ("bwd", bb), ("dbl", bd)):
+                row[name] = dict(copies=b, **_sweep_point(plan, sobek_count_graph(b), dev, (name,))[name])
+            res["table3"].append(row)
+            torch.cuda.empty_cache()
+    print(json.dumps(res), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -603,7 +728,12 @@ def main():
     ap.add_argument("--pass", dest="pass_", default="fwdbwd", choices=["fwd", "fwdbwd"])
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweeps", nargs="*", default=None, choices=["degree", "count", "table3"],
+                    help="run Sobek's scaling workloads instead of the benchmark step")
     args = ap.parse_args()
+    if args.sweeps is not None:
+        run_sweeps(argparse.Namespace(sweeps=args.sweeps or ["degree", "count", "table3"]))
+        return
     if args.warmup < 3:
         args.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "1"))

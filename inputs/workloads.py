@@ -242,3 +242,63 @@ def make_workload(cfg_id: int, n_w: int, n_nodes: Optional[int] = None,
     A = (rng.normal(size=(cfg.K, n_w)) * cfg.a_std).astype(dt)
     g = rng.normal(size=(cfg.n_nodes, c_out if c_out is not None else _irreps_dim(cfg.irreps_out))).astype(dt)
     return Workload(cfg, pos, src, dst, Y, phi, x, A, g, n_w)
+
+
+# ----------------------------------------------------------------------------- scaling graphs
+#
+# Sobek §5.1's scaling axes, on synthetic periodic positions at the density of
+# the fully connected workload (mean degree 32 at r_c = 5 A): a degree axis
+# (one set of 2048 positions, the cutoff set for the wanted mean degree) and a
+# graph-count axis (B copies of one 128-node, degree-32 graph). The pages do
+# not print the exact grids; the degrees and counts are chosen to span their
+# 8.2e3 - 2.1e6 edge range.
+
+SOBEK_RHO = 32.0 / (4.0 / 3.0 * np.pi * 5.0 ** 3)     # atoms per A^3
+SOBEK_DEGREES = (4, 8, 16, 32, 64, 128, 256, 512, 1023)
+SOBEK_COUNTS = (2, 8, 32, 128, 511)
+
+
+def _graph_features(pos, src, dst, box, r_cut, irreps_in, sh_lmax, K, n_w, c_out, a_std, seed):
+    rng = np.random.default_rng(seed)
+    vec = edge_vectors(pos, src, dst, box, True)
+    r = np.linalg.norm(vec, axis=1)
+    Y = spherical_harmonics(sh_lmax, vec).astype(np.float32)
+    phi = bessel_cutoff(r, K, r_cut).astype(np.float32)
+    n = len(pos)
+    x = rng.normal(size=(n, _irreps_dim(irreps_in))).astype(np.float32)
+    A = (rng.normal(size=(K, n_w)) * a_std).astype(np.float32)
+    g = rng.normal(size=(n, c_out)).astype(np.float32)
+    return Y, phi, x, A, g
+
+
+def sobek_degree_graph(degree: int, n_nodes: int = 2048, seed: int = 0):
+    """(positions, src, dst, box, r_cut): radius graph on fixed periodic
+    positions with the cutoff set for a mean receiver degree of `degree`."""
+    box = float((n_nodes / SOBEK_RHO) ** (1.0 / 3.0))
+    pos = np.random.default_rng(seed).uniform(0.0, box, size=(n_nodes, 3))
+    r_cut = float((3.0 * degree / (4.0 * np.pi * SOBEK_RHO)) ** (1.0 / 3.0))
+    r_cut = min(r_cut, 0.4999 * box)
+    src, dst = radius_graph(pos, box, True, r_cut)
+    return pos, src, dst, box, r_cut
+
+
+def sobek_count_graph(copies: int, n_nodes: int = 128, seed: int = 0):
+    """(positions, src, dst, box, r_cut) of `copies` disjoint copies of one
+    128-node, mean-degree-32 periodic graph (node ids offset per copy; the
+    positions of every copy are the same, each copy in its own periodic box)."""
+    box = float((n_nodes / SOBEK_RHO) ** (1.0 / 3.0))
+    pos = np.random.default_rng(seed).uniform(0.0, box, size=(n_nodes, 3))
+    src, dst = radius_graph(pos, box, True, 5.0)
+    off = np.repeat(np.arange(copies, dtype=np.int64) * n_nodes, len(src))
+    return (np.tile(pos, (copies, 1)), np.tile(src, copies) + off, np.tile(dst, copies) + off, box, 5.0)
+
+
+def sobek_workload(graph, irreps: str, sh_lmax: int, K: int, n_w: int, c_out: int, seed: int = 1):
+    """Inputs of a fully connected profile (in = out irreps) on a scaling
+    graph: Y, phi (K Bessel functions x cosine cutoff), x, A ~ N(0, 1/sqrt(K C)),
+    grad_out; float32, COO edge order."""
+    pos, src, dst, box, r_cut = graph
+    mul0 = int(irreps.split("x")[0])
+    Y, phi, x, A, g = _graph_features(pos, src, dst, box, r_cut, irreps, sh_lmax, K, n_w, c_out,
+                                      1.0 / np.sqrt(K * mul0), seed)
+    return dict(src=src, dst=dst, Y=Y, phi=phi, x=x, A=A, grad_out=g, n_nodes=len(pos))
