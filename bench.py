@@ -110,14 +110,14 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- setup
 
-def setup(cid: int, dev: str, n_nodes=None):
+def setup(cid: int, dev: str, n_nodes=None, node_order=None):
     import torch
 
     import clebsch_gordan_tensor_node_b200 as tpc
     from inputs import CONFIGS, make_workload
     c = CONFIGS[cid]
     plan = tpc.Plan(c.irreps_in, c.sh_lmax, c.irreps_out, c.K, c.mode, c.dtype, irreps_sh=c.irreps_sh)
-    wl = make_workload(cid, plan.n_w, n_nodes=n_nodes, c_out=plan.c_out)
+    wl = make_workload(cid, plan.n_w, n_nodes=n_nodes, c_out=plan.c_out, node_order=node_order)
     N, E = wl.n_nodes, wl.n_edges
     src = torch.from_numpy(wl.src.astype(np.int32)).to(dev)
     dst = torch.from_numpy(wl.dst.astype(np.int32)).to(dev)
@@ -241,11 +241,29 @@ def roofline_step(d, ms_pass, both: bool) -> dict:
     return r
 
 
+def roofline_dbl(d, ms: float) -> dict:
+    """Roofline of a double-backward step: its algorithmic flops (work model
+    pass 2) over the step time against the derived ALU peak."""
+    r = roofline(d, 2, ms)
+    r["kernel"] = "one step = the second-order program's launches"
+    t = NCU_TRAFFIC.get((d["cfg"].id, "dbl"))
+    if t is not None:
+        r["traffic"] = t[0]
+        r["traffic_source"] = f"{t[1]}: dram__bytes_read.sum + dram__bytes_write.sum, {t[2]}"
+    return r
+
+
 # DRAM bytes (read + write) per step (summed over the step's kernels) or per
 # launch of a single-kernel pass, from ncu captures of the current kernels (the
 # summaries under profiles/ give the commands); absent where no capture of the
 # current kernels exists.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    (4, "fwdbwd"): (70_358_256_640, "uvu_fwd_kernel + uvu_edge_kernel + uvu_src_kernel + reduce_slots_kernel",
+                    "profiles/uvu_step_dram_large_100k.md"),
+    (4, "fwd"): (6_991_858_176 + 434_768_640, "uvu_fwd_kernel", "profiles/uvu_step_dram_large_100k.md"),
+    (4, "dbl"): (112_633_031_680, "uvu_dbwd_recv_kernel + uvu_dbwd_edge_kernel + uvu_dbwd_src_kernel + "
+                 "reduce_slots_kernel", "profiles/uvu_step_dram_large_100k.md"),
+}
 
 
 def roofline(d, pass_: int, ms: float) -> dict:
@@ -394,8 +412,12 @@ def run_ours(args, rank, world, dist):
     c = d["cfg"]
     sampler = ClockSampler() if rank == 0 else None
     both = args.pass_ == "fwdbwd" and c.backward
+    second = args.pass_ == "dbl" and c.backward
 
     def step(marks):
+        if second:
+            dbl(d)
+            return
         fwd(d)
         if both:
             ev = torch.cuda.Event(enable_timing=True)
@@ -413,17 +435,20 @@ def run_ours(args, rank, world, dist):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": c.dtype,
            "data": "synthetic",
-           "config": {"workload": c.name, "pass": "forward+backward" if both else "forward",
+           "config": {"workload": c.name,
+                      "pass": "double backward" if second else "forward+backward" if both else "forward",
                       "n_nodes": d["N"], "n_edges": d["E"],
                       "irreps_in": c.irreps_in, "irreps_out": c.irreps_out, "sh_lmax": c.sh_lmax,
                       "n_radial": c.K, "mode": c.mode, "parallelism": f"replicas x{world}",
                       "l2": "inputs larger than L2; also flushed between steps (256 MiB write outside "
                             "the timed events)"},
-           "gpu_launches": args.steps * (d["plan"].launch_count(d["N"], 0)
+           "gpu_launches": args.steps * (d["plan"].launch_count(d["N"], 2) if second else
+                                         d["plan"].launch_count(d["N"], 0)
                                          + (d["plan"].launch_count(d["N"], 1) if both else 0)),
-           "roofline": roofline_step(d, ms_pass, both), "clocks": clocks}
+           "roofline": roofline_dbl(d, ms) if second else roofline_step(d, ms_pass, both), "clocks": clocks}
     # end to end through the public API: pinned host inputs -> device -> passes -> host results
-    res["e2e"] = e2e(d, args, both)
+    if not second:
+        res["e2e"] = e2e(d, args, both)
     if rank == 0 and not args.no_extra:
         res["workloads"] = extra_workloads(args, dev, flush, d)
         res["workspace"] = workspace_vs_edges(dev, d)
@@ -484,9 +509,14 @@ def extra_workloads(args, dev, flush, head):
 
     import clebsch_gordan_tensor_node_b200 as tpc
     out = {}
-    for cid in (1, 2, 3, 4, 5):
+    for cid in (1, 2, 3, 4, 5, "4-morton"):
         try:
-            d = head if cid == head["cfg"].id else setup(cid, dev)
+            if cid == "4-morton":
+                # the large graph with its nodes numbered along a Z-order curve:
+                # the same operator on a spatially sorted node order
+                d = setup(4, dev, node_order="morton")
+            else:
+                d = head if cid == head["cfg"].id else setup(cid, dev)
         except tpc.TpConvError as e:
             out[str(cid)] = {"skipped": str(e)}
             continue
@@ -495,10 +525,17 @@ def extra_workloads(args, dev, flush, head):
             tf, _, _ = time_steps(lambda m: fwd(d), k, 3, flush)
             ms_f = statistics.median(tf)
             rf = roofline_step(d, [ms_f], False)
-            rec = {"workload": d["cfg"].name, "n_nodes": d["N"], "n_edges": d["E"], "dtype": d["cfg"].dtype,
+            name = d["cfg"].name + (", nodes in Z-order" if cid == "4-morton" else "")
+            rec = {"workload": name, "n_nodes": d["N"], "n_edges": d["E"], "dtype": d["cfg"].dtype,
                    "fwd_ms": round(ms_f, 5), "fwd_edges_per_s": round(d["E"] / (ms_f * 1e-3), 1),
                    "fwd_roofline_frac": rf["frac"], "fwd_traffic": rf["traffic"],
                    "gpu_launches_fwd": d["plan"].launch_count(d["N"], 0)}
+            if d["cfg"].mode == "uvu":
+                # the receiver-state order (Sobek §4.2 applied to uvu), for comparison
+                d["plan"].set_schedule("receiver_state")
+                ts, _, _ = time_steps(lambda m: fwd(d), k, 3, flush)
+                d["plan"].set_schedule("streamed")
+                rec["fwd_receiver_state_ms"] = round(statistics.median(ts), 5)
             if d["cfg"].backward:
                 tb, _, _ = time_steps(lambda m: bwd(d), k, 3, flush)
                 ms_b = statistics.median(tb)
@@ -725,7 +762,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", type=int, default=4)
-    ap.add_argument("--pass", dest="pass_", default="fwdbwd", choices=["fwd", "fwdbwd"])
+    ap.add_argument("--pass", dest="pass_", default="fwdbwd", choices=["fwd", "fwdbwd", "dbl"])
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweeps", nargs="*", default=None, choices=["degree", "count", "table3"],

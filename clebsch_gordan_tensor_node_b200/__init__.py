@@ -96,6 +96,12 @@ class Plan:
         check(lib().tp_conv_plan_set_state_budget(self._h, nbytes), "tp_conv_plan_set_state_budget")
         self.state_budget = nbytes
 
+    def set_schedule(self, schedule: str) -> None:
+        """Channelwise forward order: "streamed" (default) or "receiver_state"
+        (tp_conv_plan_set_schedule)."""
+        code = {"streamed": 0, "receiver_state": 1}[schedule]
+        check(lib().tp_conv_plan_set_schedule(self._h, code), "tp_conv_plan_set_schedule")
+
     def workspace_size(self, n_nodes: int, pass_: int) -> int:
         out = ctypes.c_size_t()
         check(lib().tp_conv_workspace_size(self._h, n_nodes, pass_, ctypes.byref(out)),

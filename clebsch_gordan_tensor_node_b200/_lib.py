@@ -40,6 +40,7 @@ SIGNATURES = {
     "tp_conv_plan_cg": (c_int, [c_void_p, c_int, POINTER(c_int32), POINTER(c_int32), POINTER(c_int32),
                                 POINTER(c_double), c_int]),
     "tp_conv_plan_set_state_budget": (c_int, [c_void_p, c_size_t]),
+    "tp_conv_plan_set_schedule": (c_int, [c_void_p, c_int]),
     "tp_conv_work_model": (c_int, [c_void_p, c_int64, c_int64, c_int, POINTER(c_double), POINTER(c_double)]),
     "tp_conv_workspace_size": (c_int, [c_void_p, c_int64, c_int, POINTER(c_size_t)]),
     "tp_conv_launch_count": (c_int, [c_void_p, c_int64, c_int, POINTER(c_int)]),

@@ -29,6 +29,7 @@ UNITS = {
     "uvu_bwd.cu": 10,
     "uvw.cu": 10,
     "uvu_dbwd.cu": 10,
+    "uvu_state.cu": 2,
     "gemm.cu": 1,
     "tc_gemm.cu": 1,
     "csr.cu": 1,

@@ -103,6 +103,16 @@ template <typename T>
 int forward_uvu(const Plan& P, const void* x, const void* Y, const void* phi, const void* A,
                 const int* rowptr, const int* senders, int N, int E, void* out, int* err, cudaStream_t s) {
   UvuFwdParams<T> prm;
+  if (P.schedule == TP_SCHED_RECEIVER_STATE) {
+    std::memset(&prm, 0, sizeof(prm));
+    prm.x = (const T*)x; prm.Y = (const T*)Y; prm.phi = (const T*)phi; prm.A = (const T*)A;
+    prm.rowptr = rowptr; prm.senders = senders; prm.out = (T*)out; prm.err = err;
+    prm.N = N; prm.E = E; prm.K = P.K; prm.c_in = P.c_in; prm.c_out = P.c_out; prm.dim_y = P.dim_y;
+    prm.n_w = (int)P.n_w;
+    copy_tables(prm, P.dbl_out_tiles, P.dbl_paths_by_out);
+    cudaError_t e = launch_uvu_state_fwd<T>(prm, P.prof, s);
+    return e == cudaSuccess ? TP_OK : cuda_fail(e, "uvu receiver-state forward launch");
+  }
   prm.x = (const T*)x; prm.Y = (const T*)Y; prm.phi = (const T*)phi; prm.A = (const T*)A;
   prm.rowptr = rowptr; prm.senders = senders; prm.out = (T*)out; prm.err = err;
   prm.N = N; prm.E = E; prm.K = P.K; prm.c_in = P.c_in; prm.c_out = P.c_out; prm.dim_y = P.dim_y;
@@ -700,6 +710,20 @@ int tp_conv_plan_set_state_budget(tp_plan_t plan, size_t bytes) {
     return fail(TP_EINVAL, "state budget " + std::to_string(bytes) + " bytes is below one node's state (" +
                                std::to_string(one) + " bytes)");
   P.state_budget = bytes;
+  return TP_OK;
+}
+
+int tp_conv_plan_set_schedule(tp_plan_t plan, int schedule) {
+  if (!plan) return fail(TP_EINVAL, "NULL plan");
+  Plan& P = plan->p;
+  if (schedule != TP_SCHED_STREAMED && schedule != TP_SCHED_RECEIVER_STATE)
+    return fail(TP_EINVAL, "schedule must be TP_SCHED_STREAMED or TP_SCHED_RECEIVER_STATE");
+  if (P.mode != TP_UVU) return schedule == TP_SCHED_RECEIVER_STATE ? TP_OK
+                                                                  : fail(TP_EUNSUPPORTED, "fully connected plans "
+                                                                                          "use the receiver state");
+  if (schedule == TP_SCHED_RECEIVER_STATE && (P.K > 8 || P.prof > 3 || !P.dbl_ok))
+    return fail(TP_EUNSUPPORTED, "the receiver-state uvu forward is compiled for K <= 8 and degrees <= 4");
+  P.schedule = schedule;
   return TP_OK;
 }
 

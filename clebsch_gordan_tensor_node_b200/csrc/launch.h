@@ -8,6 +8,11 @@
 
 namespace tpc {
 
+// Channelwise forward in the receiver-factorised order (uvu_state.cu): 32-channel
+// tiles of the output blocks, K <= 8, degree profiles 0-3.
+template <typename T>
+cudaError_t launch_uvu_state_fwd(const UvuFwdParams<T>& p, int prof, cudaStream_t s);
+
 // Edge pass of the uvu backward: radial width KP, gather width V, degree profile.
 template <typename T>
 cudaError_t launch_uvu_edge_for(const Plan& P, const UvuEdgeParams<T>& p, cudaStream_t s) {

@@ -26,6 +26,7 @@ constexpr size_t kUvwChunkBytes = size_t(1) << 30;
 struct Plan {
   int mode = 0;     // 0 uvu, 1 uvw
   bool per_path = false;    // uvu with one output block per path
+  int schedule = 0;         // uvu forward: 0 streamed (Sobek §3.1), 1 receiver state (Sobek §4.2)
   int dtype = 0;    // 0 f32, 1 f64
   int K = 0, KP = 0, CPL = 1, sh_lmax = 0, lmax = 0;
   int fwd_CPL = 1;          // channels per lane of the forward kernel

@@ -62,6 +62,7 @@ typedef struct tp_plan_s* tp_plan_t;
 
 enum tp_mode { TP_UVU = 0, TP_UVW = 1, TP_UVU_PATHS = 2 };
 enum tp_dtype { TP_F32 = 0, TP_F64 = 1 };
+enum tp_schedule { TP_SCHED_STREAMED = 0, TP_SCHED_RECEIVER_STATE = 1 };
 enum tp_status {
   TP_OK = 0,
   TP_EINVAL = -1,         /* bad argument (null pointer, size, alignment, string) */
@@ -155,6 +156,19 @@ int tp_conv_plan_cg(tp_plan_t plan, int index, int32_t* m1, int32_t* m2, int32_t
  * (the message gives that size). Channelwise (uvu) plans keep no state
  * chunks and accept any value without effect. */
 int tp_conv_plan_set_state_budget(tp_plan_t plan, size_t bytes);
+
+/* Evaluation order of the channelwise forward. TP_SCHED_STREAMED (default):
+ * Sobek §3.1, the scalar w = phi A formed per edge, path and channel and
+ * consumed at once. TP_SCHED_RECEIVER_STATE: Sobek §4.2 (Eqs. 32-35) applied to
+ * uvu, the receiver state S_i = sum_e phi_e (outer) C(x_j, Y_e) per path and
+ * channel kept in registers over the receiver's edges and mixed with A once per
+ * receiver; it costs nnz + K (2 l3 + 1) FMAs per edge and channel against
+ * K + nnz + (2 l3 + 1) and exists to compare the two orders. Both give the
+ * same result up to rounding order. Fully connected plans always use the
+ * receiver state (TP_SCHED_STREAMED is TP_EUNSUPPORTED for them). Errors:
+ * TP_EINVAL (unknown schedule), TP_EUNSUPPORTED (receiver state with K > 8 or
+ * degrees above 4). Host only. */
+int tp_conv_plan_set_schedule(tp_plan_t plan, int schedule);
 
 /* Algorithmic work of one pass (0 forward, 1 backward, 2 double backward) on
  * N nodes and E edges: flops (FMA = 2) of the streamed schedule and compulsory

@@ -121,6 +121,17 @@ def _positions(cfg: Config, rng: np.random.Generator) -> np.ndarray:
     return rng.uniform(0.0, cfg.box, size=(cfg.n_nodes, 3))
 
 
+def morton_order(pos: np.ndarray, box: float, bits: int = 10) -> np.ndarray:
+    """Permutation that sorts points along a Z-order (Morton) curve of the box:
+    each coordinate quantised to `bits` bits, the bits interleaved x, y, z."""
+    q = np.clip((pos / box * (1 << bits)).astype(np.int64), 0, (1 << bits) - 1)
+    code = np.zeros(len(pos), np.int64)
+    for b in range(bits):
+        for d in range(3):
+            code |= ((q[:, d] >> b) & 1) << (3 * b + d)
+    return np.argsort(code, kind="stable")
+
+
 def radius_graph(pos: np.ndarray, box: float, periodic: bool, r_cut: float):
     """All ordered pairs (src, dst), src != dst, |r_dst - r_src| < r_cut (min. image)."""
     if periodic:
@@ -208,7 +219,8 @@ class Workload:
 
 
 def make_workload(cfg_id: int, n_w: int, n_nodes: Optional[int] = None,
-                  edge_keep: Optional[float] = None, c_out: Optional[int] = None) -> Workload:
+                  edge_keep: Optional[float] = None, c_out: Optional[int] = None,
+                  node_order: Optional[str] = None) -> Workload:
     """Build workload ``cfg_id``.
 
     n_w (the weight count of the operator's path layout) and c_out (the output
@@ -216,6 +228,9 @@ def make_workload(cfg_id: int, n_w: int, n_nodes: Optional[int] = None,
     this module stays free of the operator's path rules. ``n_nodes`` shrinks a
     periodic workload at fixed density (for fast tests); ``edge_keep`` keeps a
     seeded fraction of the edges (for workspace-versus-edge-count checks).
+    ``node_order="morton"`` numbers the nodes along a Z-order curve of their
+    positions (a spatially sorted variant; the default keeps generation order,
+    which is spatially random).
     """
     cfg = CONFIGS[cfg_id]
     if n_nodes is not None and n_nodes != cfg.n_nodes:
@@ -229,6 +244,10 @@ def make_workload(cfg_id: int, n_w: int, n_nodes: Optional[int] = None,
         pos = _positions(CONFIGS[cfg.positions_from], np.random.default_rng(cfg.positions_from))
     else:
         pos = _positions(cfg, rng)
+    if node_order == "morton":
+        pos = pos[morton_order(pos, cfg.box)]
+    elif node_order is not None:
+        raise ValueError(f"unknown node order {node_order!r}")
     src, dst = radius_graph(pos, cfg.box, cfg.periodic, cfg.r_cut)
     if edge_keep is not None:
         keep = np.random.default_rng(1000 + cfg.id).random(len(src)) < edge_keep

@@ -165,3 +165,19 @@ def test_per_path_outputs_match_lunatp_table1():
             tot[(p.l3, p.p3)] = tot.get((p.l3, p.p3), 0) + p.mul_in
         assert tot == gold[case], case
         assert len(outs) == plan.n_paths
+
+
+def test_schedule_option():
+    """The receiver-state order is accepted for channelwise plans within its
+    compiled limits and rejected outside them."""
+    uvu = tpc.Plan("8x0e+8x1o", 1, "8x0e+8x1o", 8, "uvu", "f32")
+    uvu.set_schedule("receiver_state")
+    uvu.set_schedule("streamed")
+    wide = tpc.Plan("8x0e", 1, "8x0e+8x1o", 16, "uvu", "f32")
+    with pytest.raises(tpc.TpConvError) as ei:
+        wide.set_schedule("receiver_state")
+    assert ei.value.status == -2
+    uvw = tpc.Plan("8x0e", 1, "8x0e+8x1o", 8, "uvw", "f32")
+    uvw.set_schedule("receiver_state")
+    with pytest.raises(tpc.TpConvError):
+        uvw.set_schedule("streamed")
