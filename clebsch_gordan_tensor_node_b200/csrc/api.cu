@@ -171,9 +171,9 @@ int double_backward_uvu(const Plan& P, const void* const* in, const int* const* 
   p.err = err;
   p.N = N; p.E = E; p.K = P.K; p.c_in = P.c_in; p.c_out = P.c_out; p.dim_y = P.dim_y; p.n_w = (int)P.n_w;
   const bool k8 = P.KP == 8;
-  // receiver pass: m_dot
+  // receiver pass: m_dot (one channel per lane, 32-channel tiles)
   copy_tables(p, P.dbl_out_tiles, P.dbl_paths_by_out);
-  cudaError_t e = k8 ? launch_uvu_dbwd_recv<T, 8>(p, P.prof, s) : launch_uvu_dbwd_recv<T, 16>(p, P.prof, s);
+  cudaError_t e = k8 ? launch_uvu_dbwd_recv<T, 8, 1>(p, P.prof, s) : launch_uvu_dbwd_recv<T, 16, 1>(p, P.prof, s);
   if (e != cudaSuccess) return cuda_fail(e, "double backward receiver pass");
   // edge pass: phi_bar_dot, Y_bar_dot
   std::memset(p.paths, 0, sizeof(p.paths));
@@ -186,9 +186,9 @@ int double_backward_uvu(const Plan& P, const void* const* in, const int* const* 
     e = k8 ? launch_uvu_dbwd_edge<T, 8, 1>(p, P.prof, s) : launch_uvu_dbwd_edge<T, 16, 1>(p, P.prof, s);
   if (e != cudaSuccess) return cuda_fail(e, "double backward edge pass");
   // source pass: x_bar_dot and the A_bar_dot slot partials, then their sum
-  copy_tables(p, P.dbl_in_tiles, P.dbl_paths_by_in);
   p.n_slots = uvu_src_slots(P, N);
-  e = k8 ? launch_uvu_dbwd_src<T, 8>(p, P.prof, s) : launch_uvu_dbwd_src<T, 16>(p, P.prof, s);
+  copy_tables(p, P.dbl_in_tiles, P.dbl_paths_by_in);
+  e = k8 ? launch_uvu_dbwd_src<T, 8, 1>(p, P.prof, s) : launch_uvu_dbwd_src<T, 16, 1>(p, P.prof, s);
   if (e != cudaSuccess) return cuda_fail(e, "double backward source pass");
   e = launch_reduce_slots<T>((const T*)ws, (T*)out[4], p.n_slots, (long long)P.K * P.n_w, s);
   return e == cudaSuccess ? TP_OK : cuda_fail(e, "double backward A_bar reduction");

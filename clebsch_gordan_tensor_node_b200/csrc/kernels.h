@@ -24,11 +24,11 @@ cudaError_t launch_reduce_slots(const T* part, T* out, int n_slots, long long n,
 // second-order program of the channelwise path: receiver pass (m_dot), edge
 // pass (phi_bar_dot, Y_bar_dot; V channels per gather) and source pass
 // (x_bar_dot, A_bar_dot slot partials, zeroed first)
-template <typename T, int KP>
+template <typename T, int KP, int CPL>
 cudaError_t launch_uvu_dbwd_recv(const UvuDbwdParams<T>& p, int prof, cudaStream_t s);
 template <typename T, int KP, int V>
 cudaError_t launch_uvu_dbwd_edge(const UvuDbwdParams<T>& p, int prof, cudaStream_t s);
-template <typename T, int KP>
+template <typename T, int KP, int CPL>
 cudaError_t launch_uvu_dbwd_src(const UvuDbwdParams<T>& p, int prof, cudaStream_t s);
 
 template <typename T, int KP, int DIR>

@@ -442,8 +442,11 @@ constexpr bool wide_ok() { return std::is_same<T, float>::value && KP == 8; }
 
 }  // namespace
 
-template <typename T, int KP>
+// One channel per lane (CPL = 1): wider lanes measured slower (register spills
+// in the source pass, no gain in the receiver pass).
+template <typename T, int KP, int CPL>
 cudaError_t launch_uvu_dbwd_recv(const UvuDbwdParams<T>& p, int prof, cudaStream_t s) {
+  static_assert(CPL == 1, "the second-order passes run one channel per lane");
   const long long tasks = (long long)p.N * p.n_tiles;
   if (tasks == 0) return cudaSuccess;
   const unsigned blocks = (unsigned)((tasks + kDbWarps - 1) / kDbWarps);
@@ -470,8 +473,9 @@ cudaError_t launch_uvu_dbwd_edge(const UvuDbwdParams<T>& p0, int prof, cudaStrea
   });
 }
 
-template <typename T, int KP>
+template <typename T, int KP, int CPL>
 cudaError_t launch_uvu_dbwd_src(const UvuDbwdParams<T>& p, int prof, cudaStream_t s) {
+  static_assert(CPL == 1, "the second-order passes run one channel per lane");
   cudaError_t err = cudaMemsetAsync(p.apart, 0, sizeof(T) * (size_t)p.n_slots * p.K * p.n_w, s);
   if (err != cudaSuccess) return err;
   if (p.n_slots == 0 || p.n_tiles == 0 || p.N == 0) return cudaSuccess;
@@ -482,8 +486,10 @@ cudaError_t launch_uvu_dbwd_src(const UvuDbwdParams<T>& p, int prof, cudaStream_
   });
 }
 
-#define TPC_INST_R(T, KP) template cudaError_t launch_uvu_dbwd_recv<T, KP>(const UvuDbwdParams<T>&, int, cudaStream_t);
-#define TPC_INST_S(T, KP) template cudaError_t launch_uvu_dbwd_src<T, KP>(const UvuDbwdParams<T>&, int, cudaStream_t);
+#define TPC_INST_R(T, KP) \
+  template cudaError_t launch_uvu_dbwd_recv<T, KP, 1>(const UvuDbwdParams<T>&, int, cudaStream_t);
+#define TPC_INST_S(T, KP) \
+  template cudaError_t launch_uvu_dbwd_src<T, KP, 1>(const UvuDbwdParams<T>&, int, cudaStream_t);
 #define TPC_INST_E(T, KP, V) \
   template cudaError_t launch_uvu_dbwd_edge<T, KP, V>(const UvuDbwdParams<T>&, int, cudaStream_t);
 #if TPC_WANT(0)
