@@ -422,12 +422,12 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
       P.uvw_in.push_back(b);
     }
     P.sa_row_elems = sa_off;
-    // tensor-core mixing: fp32, at most 64 channels per block (one 128 x 64 tile
-    // pipeline fits shared memory), state rows whose width is a multiple of 4
-    // (16-byte TMA strides)
+    // tensor-core mixing: fp32, at most 256 channels per block (one 128 x N
+    // accumulator in tensor memory; the ring shrinks to fit shared memory), state
+    // rows whose width is a multiple of 4 (16-byte TMA strides)
     P.uvw_tc = dtype == TP_F32;
-    for (auto& b : P.uvw_out) P.uvw_tc = P.uvw_tc && b.mul_own <= 64 && b.dcols % 4 == 0;
-    for (auto& b : P.uvw_in) P.uvw_tc = P.uvw_tc && b.mul_own <= 64 && b.dcols % 4 == 0;
+    for (auto& b : P.uvw_out) P.uvw_tc = P.uvw_tc && b.mul_own <= 256 && b.dcols % 4 == 0;
+    for (auto& b : P.uvw_in) P.uvw_tc = P.uvw_tc && b.mul_own <= 256 && b.dcols % 4 == 0;
     const size_t bsz2 = dtype == TP_F32 ? 4 : 8;
     if ((size_t)std::max(P.s_row_elems, P.sa_row_elems) * bsz2 > P.state_budget) {
       msg = "one node's uvw state exceeds the state chunk budget";

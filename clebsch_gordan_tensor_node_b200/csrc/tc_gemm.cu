@@ -14,7 +14,7 @@
 // relative). Bt is split once by the packing kernel; X is split in shared memory.
 //
 // One CTA (4 warps) owns 128 rows and all N (<= 256, padded to 16) columns;
-// the fp32 accumulator lives in tensor memory. K runs through a 4-stage
+// the fp32 accumulator lives in tensor memory. K runs through a 2- to 4-stage
 // shared-memory pipeline in 32-wide tiles:
 //   warp 0 (one lane): TMA producer -- cp.async.bulk.tensor loads of the raw X
 //            tile [128 x 32] and the Bt_hi / Bt_lo tiles [N x 32], 128-byte
@@ -39,7 +39,7 @@ namespace {
 
 constexpr int TM = 128;        // rows per CTA (tensor-memory lanes)
 constexpr int KT = 32;         // K per stage (one 128-byte swizzle row of fp32)
-constexpr int NS = 4;          // pipeline stages
+constexpr int kMaxStages = 4;  // pipeline stages for output blocks of up to 64 channels
 constexpr long long kSpinLimit = 1ll << 22;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -117,6 +117,9 @@ struct Stage {
   float* bl;  // Bt_lo tile
 };
 
+// NS: pipeline stages; wider output blocks (npmax up to 256) take fewer stages so
+// that the ring stays within shared memory.
+template <int NS>
 __global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__ TcBatch tb, int npmax, int* err) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ int fail_flag;
@@ -324,18 +327,29 @@ bool tc_make_map(CUtensorMap* map, const float* base, long long rows, long long 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-size_t tc_smem_bytes(int npmax) {
-  return 1024 + (size_t)NS * (2 * TM * KT * 4 + 2 * (size_t)npmax * KT * 4) + (3 * NS + 1) * 8 + 16;
+size_t tc_smem_bytes(int npmax, int ns) {
+  return 1024 + (size_t)ns * (2 * TM * KT * 4 + 2 * (size_t)npmax * KT * 4) + (3 * ns + 1) * 8 + 16;
 }
 
+template <int NS>
+cudaError_t launch_tc_ns(const TcBatch& tb, int n_prob, int max_m, int npmax, int* err, cudaStream_t s) {
+  const size_t smem = tc_smem_bytes(npmax, NS);
+  static SmemLimit limit;
+  if (cudaError_t e = limit.ensure((const void*)tc_gemm_kernel<NS>, smem); e != cudaSuccess) return e;
+  dim3 grid((max_m + TM - 1) / TM, n_prob);
+  tc_gemm_kernel<NS><<<grid, 128, smem, s>>>(tb, npmax, err);
+  return cudaGetLastError();
+}
+
+// Output blocks up to 256 channels (padded to 16): the deepest ring that fits
+// 227 KiB of shared memory, 4 stages up to 64 channels, 3 up to 128, 2 up to 256.
 cudaError_t launch_gemm_tc(const TcBatch& tb, int n_prob, int max_m, int npmax, int* err, cudaStream_t s) {
   if (n_prob == 0 || max_m == 0) return cudaSuccess;
-  const size_t smem = tc_smem_bytes(npmax);
-  static SmemLimit limit;
-  if (cudaError_t e = limit.ensure((const void*)tc_gemm_kernel, smem); e != cudaSuccess) return e;
-  dim3 grid((max_m + TM - 1) / TM, n_prob);
-  tc_gemm_kernel<<<grid, 128, smem, s>>>(tb, npmax, err);
-  return cudaGetLastError();
+  if (npmax > 256) return cudaErrorInvalidValue;
+  const size_t cap = 227 * 1024;
+  if (tc_smem_bytes(npmax, kMaxStages) <= cap) return launch_tc_ns<kMaxStages>(tb, n_prob, max_m, npmax, err, s);
+  if (tc_smem_bytes(npmax, 3) <= cap) return launch_tc_ns<3>(tb, n_prob, max_m, npmax, err, s);
+  return launch_tc_ns<2>(tb, n_prob, max_m, npmax, err, s);
 }
 
 }  // namespace tpc

@@ -171,38 +171,41 @@ __device__ __forceinline__ void sbuild_path(const UvwSParams<T>& p, const UvwBlo
       __syncthreads();
     }
     T* dst = p.S + (size_t)p.nr_alloc * bd.s_off + (size_t)(r - p.r0) * DO * bd.dcols + pd.col_off;
-    if constexpr (kTC) {
-      // C fragment: rows q = gid, gid + 8; columns u = 8 warp + 2 tig, + 1
-      const int u = c0 + warp * 8 + 2 * tig;
+    // the accumulate choice is taken once, outside the unrolled store loops
+    auto store = [&](auto Acc) {
+      constexpr bool kAcc = decltype(Acc)::value;
+      if constexpr (kTC) {
+        // C fragment: rows q = gid, gid + 8; columns u = 8 warp + 2 tig, + 1
+        const int u = c0 + warp * 8 + 2 * tig;
 #pragma unroll
-      for (int m = 0; m < DO; ++m) {
+        for (int m = 0; m < DO; ++m) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int q = gid + 8 * h;
-          if (q >= p.K) continue;
-          T* row = dst + (size_t)m * bd.dcols + (size_t)q * gmul;
-          if (p.accumulate) {
-            if (u < gmul) row[u] += acc[m][2 * h];
-            if (u + 1 < gmul) row[u + 1] += acc[m][2 * h + 1];
-          } else {
-            if (u < gmul) row[u] = acc[m][2 * h];
-            if (u + 1 < gmul) row[u + 1] = acc[m][2 * h + 1];
+          for (int h = 0; h < 2; ++h) {
+            const int q = gid + 8 * h;
+            if (q >= p.K) continue;
+            T* row = dst + (size_t)m * bd.dcols + (size_t)q * gmul;
+            if (u < gmul) row[u] = kAcc ? row[u] + acc[m][2 * h] : acc[m][2 * h];
+            if (u + 1 < gmul) row[u + 1] = kAcc ? row[u + 1] + acc[m][2 * h + 1] : acc[m][2 * h + 1];
+          }
+        }
+      } else if (act) {
+#pragma unroll
+        for (int q = 0; q < KQ; ++q) {
+          const int qq = warp * KQ + q;
+          if (qq < p.K) {
+#pragma unroll
+            for (int m = 0; m < DO; ++m) {
+              T* o = dst + (size_t)m * bd.dcols + (size_t)qq * gmul + cl;
+              *o = kAcc ? *o + Sr[q][m] : Sr[q][m];
+            }
           }
         }
       }
-    } else if (act) {
-#pragma unroll
-      for (int q = 0; q < KQ; ++q) {
-        const int qq = warp * KQ + q;
-        if (qq < p.K) {
-#pragma unroll
-          for (int m = 0; m < DO; ++m) {
-            T* o = dst + (size_t)m * bd.dcols + (size_t)qq * gmul + cl;
-            *o = p.accumulate ? *o + Sr[q][m] : Sr[q][m];
-          }
-        }
-      }
-    }
+    };
+    if (p.accumulate)
+      store(std::true_type{});
+    else
+      store(std::false_type{});
   }
 }
 
