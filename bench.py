@@ -241,6 +241,40 @@ def roofline_step(d, ms_pass, both: bool) -> dict:
     return r
 
 
+def tensor_aware_peak_tflops():
+    """fp32-exact mixing on the tensor cores: three TF32 products per output
+    (3xTF32 split); TF32 runs at half the measured dense bf16 rate (the
+    nominal 1.1 vs 2.25 PFLOP/s ratio). From MEASURED_PEAKS.json, else the
+    fallback burst figure of 1.59 PFLOP/s bf16."""
+    p = measured_peaks()
+    bf16 = float(p["bf16_tflops"]) if p and "bf16_tflops" in p else 1590.0
+    return bf16 / 2.0 / 3.0
+
+
+def uvw_mixing_flops(plan, n_nodes: int, pass_: int) -> float:
+    """Flops of the channel-mixing products (Sobek Eqs. 34-36): per receiver and
+    path 2 (2 l3 + 1) K C_in C_out each; forward one product, backward the
+    two of Eq. 36 plus the source mixing of x_bar."""
+    r = 0.0
+    for p in plan.paths():
+        r += 2.0 * (2 * p.l3 + 1) * plan.n_radial * p.mul_in * p.mul_out
+        if pass_ == 1:
+            r += 2.0 * 2 * (2 * p.l3 + 1) * plan.n_radial * p.mul_in * p.mul_out \
+                 + 2.0 * (2 * p.l1 + 1) * plan.n_radial * p.mul_in * p.mul_out
+    return r * n_nodes
+
+
+def tensor_aware_frac(d, pass_: int, ms: float):
+    """Roofline fraction of a fully connected pass with the mixing products at
+    the 3xTF32 tensor rate and the rest at the FP32 ALU peak."""
+    if d["cfg"].mode != "uvw":
+        return None
+    flops, _ = d["plan"].work_model(d["N"], d["E"], pass_)
+    mix = uvw_mixing_flops(d["plan"], d["N"], pass_)
+    t = (flops - mix) / (alu_peak("f32") * 1e12) + mix / (tensor_aware_peak_tflops() * 1e12)
+    return round(t / (ms * 1e-3), 4)
+
+
 def roofline_dbl(d, ms: float) -> dict:
     """Roofline of a double-backward step: its algorithmic flops (work model
     pass 2) over the step time against the derived ALU peak."""
@@ -529,6 +563,7 @@ def extra_workloads(args, dev, flush, head):
             rec = {"workload": name, "n_nodes": d["N"], "n_edges": d["E"], "dtype": d["cfg"].dtype,
                    "fwd_ms": round(ms_f, 5), "fwd_edges_per_s": round(d["E"] / (ms_f * 1e-3), 1),
                    "fwd_roofline_frac": rf["frac"], "fwd_traffic": rf["traffic"],
+                   "fwd_roofline_frac_tensor_aware": tensor_aware_frac(d, 0, ms_f),
                    "gpu_launches_fwd": d["plan"].launch_count(d["N"], 0)}
             if d["cfg"].mode == "uvu":
                 # the receiver-state order (Sobek §4.2 applied to uvu), for comparison
@@ -543,6 +578,7 @@ def extra_workloads(args, dev, flush, head):
                 rec.update({"bwd_ms": round(ms_b, 5),
                             "fwd_bwd_edges_per_s": round(d["E"] / ((ms_f + ms_b) * 1e-3), 1),
                             "bwd_roofline_frac": rb["passes"]["bwd"]["frac"],
+                            "bwd_roofline_frac_tensor_aware": tensor_aware_frac(d, 1, ms_b),
                             "fwd_bwd_roofline_frac": rb["frac"],
                             "workspace_bwd_bytes": d["plan"].workspace_size(d["N"], 1),
                             "gpu_launches_bwd": d["plan"].launch_count(d["N"], 1)})
