@@ -148,7 +148,7 @@ int backward_uvu(const Plan& P, const void* x, const void* Y, const void* phi, c
   sp.gx = (T*)gx; sp.apart = (T*)ws; sp.err = err;
   sp.N = N; sp.E = E; sp.K = P.K; sp.c_in = P.c_in; sp.c_out = P.c_out; sp.dim_y = P.dim_y;
   sp.n_w = (int)P.n_w;
-  sp.n_slots = uvu_src_slots(P, N);
+  sp.n_slots = 1 << 30;   // the workspace holds the partition's slots
   copy_tables(sp, P.in_tiles, P.paths_by_in);
   e = launch_uvu_src_for<T>(P, sp, s);
   if (e != cudaSuccess) return cuda_fail(e, "uvu source pass launch");

@@ -27,8 +27,11 @@ cudaError_t launch_uvu_edge_for(const Plan& P, const UvuEdgeParams<T>& p, cudaSt
 }
 
 // Source pass of the uvu backward: radial width KP, channels per lane, profile.
+// On entry p.n_slots is the most A_bar partial slots the caller's buffer holds;
+// on return it is the number the launch used (the tile partition's).
 template <typename T>
 cudaError_t launch_uvu_src_for(const Plan& P, UvuSrcParams<T>& p, cudaStream_t s) {
+  p.n_slots = uvu_src_partition(P, p.N, p.n_slots, p.tile_cta);
   p.cy_stride = P.src_cy_stride;
   p.chunk = P.src_chunk;
   p.warp_smem = P.src_warp_smem;

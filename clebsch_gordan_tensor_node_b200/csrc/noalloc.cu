@@ -92,7 +92,7 @@ int run(const Plan& P, const void* x, const void* Y, const void* phi, const void
   // call's contents), then accumulates into them
   e = launch_uvu_src_for<T>(P, sp, s);
   if (e != cudaSuccess) return set_error_message(TP_ECUDA, std::string("source pass: ") + cudaGetErrorString(e));
-  e = launch_reduce_slots<T>((const T*)scratch, (T*)gA, slots, (long long)P.K * P.n_w, s);
+  e = launch_reduce_slots<T>((const T*)scratch, (T*)gA, sp.n_slots, (long long)P.K * P.n_w, s);
   if (e != cudaSuccess) return set_error_message(TP_ECUDA, std::string("grad_A reduction: ") + cudaGetErrorString(e));
   return TP_OK;
 }
@@ -142,7 +142,7 @@ extern "C" int tp_conv_backward_noalloc(tp_plan_t plan, const void* x, const voi
   if (st) return st;
   void* scratch = nullptr;
   if ((st = scratch_address(&scratch))) return st;
-  const int slots = (int)std::min<size_t>((size_t)uvu_src_slots(P, n_nodes), fit);
+  const int slots = (int)std::min<size_t>(fit, 1 << 30);   // the source pass uses at most this many
   return P.dtype == TP_F32
              ? run<float>(P, x, Y, phi, A, rowptr, senders, colptr, srcedge, srcrecv, grad_out, (int)n_nodes,
                           (int)n_edges, grad_x, grad_Y, grad_phi, grad_A, scratch, slots, err, s)

@@ -309,8 +309,9 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
   }
   // the same staging for the source pass of the backward (paths by input block)
   P.src_cy_stride = vw;
+  P.in_tile_cost.clear();
   for (const TileD& t : P.in_tiles) {
-    int off = 0;
+    int off = 0, cost = 0;
     for (int k = t.pbeg; k < t.pend; ++k) {
       PathD& d = P.paths_by_in[k];
       auto e = real_cg_sparse(d.l1, d.l2, d.l3);
@@ -320,8 +321,13 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
       pairs.erase(std::unique(pairs.begin(), pairs.end()), pairs.end());
       d.cy_off = off;
       off += ((int)pairs.size() + vw - 1) / vw * vw;
+      // per edge: the adjoint contraction (one FMA per (m1, m3) pair), x_bar and
+      // h (2 per m1), w and the A_bar update (K each) and the radial row, the
+      // m_bar components read from the ring
+      cost += (int)pairs.size() + 2 * (2 * d.l1 + 1) + 3 * P.K + (2 * d.l3 + 1);
     }
     P.src_cy_stride = std::max(P.src_cy_stride, off);
+    P.in_tile_cost.push_back(std::max(1, cost));
   }
   // source pass: per warp, the staged chunk (receivers, radial rows, cY) and an
   // m_bar copy ring of two groups of ring_g edges (every component of the
@@ -470,11 +476,57 @@ int uvu_src_slots(const Plan& p, long long n_nodes) {
   return (int)s;
 }
 
+int uvu_src_partition(const Plan& p, long long n_nodes, long long max_slots, int* cta) {
+  const int t = (int)p.in_tiles.size();
+  if (t == 0) {
+    if (cta) cta[0] = 0;
+    return 0;
+  }
+  const int bsz = p.dtype == TP_F32 ? 4 : 8;
+  const long long w = src_warps_for(bsz);
+  const long long grid = std::max<long long>(t, (long long)kSMs * ctas_per_sm_for(bsz));
+  const long long cap = std::max<long long>(1, (n_nodes + w - 1) / w);   // CTAs with a source for every warp
+  double tot = 0;
+  for (int k = 0; k < t; ++k) tot += p.in_tile_cost[k];
+  // proportional shares rounded down (at least one CTA each), then the CTAs
+  // left over one at a time to the tile with the most cost per CTA
+  std::vector<long long> c(t);
+  long long used = 0;
+  for (int k = 0; k < t; ++k) {
+    c[k] = std::min(cap, std::max<long long>(1, (long long)(grid * (p.in_tile_cost[k] / tot))));
+    used += c[k];
+  }
+  while (used < grid) {
+    int best = -1;
+    double bv = 0;
+    for (int k = 0; k < t; ++k) {
+      const double v = p.in_tile_cost[k] / (double)c[k];
+      if (c[k] < cap && v > bv) {
+        bv = v;
+        best = k;
+      }
+    }
+    if (best < 0) break;
+    ++c[best];
+    ++used;
+  }
+  long long slots = 0;
+  for (int k = 0; k < t; ++k) slots = std::max(slots, c[k] * w);
+  slots = std::max<long long>(1, std::min(slots, max_slots));
+  if (cta) {
+    cta[0] = 0;
+    for (int k = 0; k < t; ++k) cta[k + 1] = cta[k] + (int)c[k];
+  }
+  return (int)slots;
+}
+
 size_t workspace_bytes(const Plan& p, long long n_nodes, int pass) {
   const size_t b = p.dtype == TP_F32 ? 4 : 8;
   size_t bytes = 0;
   if (p.mode == TP_UVU) {
-    if (pass >= 1) bytes = (size_t)uvu_src_slots(p, n_nodes) * p.K * p.n_w * b;
+    // first order: the source pass's slots; second order: its own source pass
+    if (pass == 1) bytes = (size_t)uvu_src_partition(p, n_nodes, 1LL << 40, nullptr) * p.K * p.n_w * b;
+    if (pass >= 2) bytes = (size_t)uvu_src_slots(p, n_nodes) * p.K * p.n_w * b;
   } else {
     // packed A (forward operand; plus adjoint operand and packed A_bar in the
     // backward), each 256-byte aligned, and one (forward) or two (backward)

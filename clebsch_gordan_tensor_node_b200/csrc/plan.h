@@ -45,6 +45,7 @@ struct Plan {
   std::vector<PathD> paths_by_out;
   std::vector<TileD> in_tiles;    // (input block, channel tile), paths_by_in ranges
   std::vector<PathD> paths_by_in;
+  std::vector<int> in_tile_cost;  // source pass: estimated warp instructions per edge of each in_tiles entry
   std::vector<PathD> paths_canon;
   // second-order program: 32-channel tiles of the output and input blocks
   std::vector<TileD> dbl_out_tiles;
@@ -78,8 +79,16 @@ int uvw_chunk_rows(const Plan& p, long long n_nodes, int dir);
 int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_radial, int mode,
               int dtype, Plan& out, std::string& msg, const int* sh_parity = nullptr);
 
-// Slots of the source pass's A_bar partial buffer (fixed per (plan, N)).
+// Slots of the double-backward source pass's A_bar partial buffer (fixed per (plan, N)).
 int uvu_src_slots(const Plan& p, long long n_nodes);
+
+// CTAs of the first-order source pass, dealt to the input-block tiles in
+// proportion to their per-edge cost (one wave; at least one CTA per tile, and
+// no more warps per tile than sources): tile t gets CTAs [cta[t], cta[t + 1])
+// when cta (n_tiles + 1 entries) is not null. Returns the A_bar partial slots,
+// the largest per-tile warp count capped at max_slots (each warp owns one slot
+// of its tile's columns and serves every slots-th source).
+int uvu_src_partition(const Plan& p, long long n_nodes, long long max_slots, int* cta);
 
 // Bytes of workspace for pass 0 (forward) or 1 (backward) at n_nodes receivers.
 size_t workspace_bytes(const Plan& p, long long n_nodes, int pass);

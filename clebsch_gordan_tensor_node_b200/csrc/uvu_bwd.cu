@@ -215,9 +215,14 @@ uvu_edge_kernel(const __grid_constant__ UvuEdgeParams<T> p) {
 // block b, channel tile); per chunk of up to 32 outgoing edges, lanes first
 // stage each edge's receiver, radial row and the cY values of every path of b
 // in shared memory; then every path sweeps the chunk with A in registers and
-// the receivers' m_bar rows arriving through an asynchronous copy ring. x_bar_j accumulates in registers
-// in one fixed order; the same sweep forms h = <x_j, t'> and adds phi h to the
-// warp's slot of the A_bar partial buffer after each path.
+// the receivers' m_bar rows arriving through an asynchronous copy ring. x_bar_j
+// accumulates in registers in one fixed order; the same sweep forms
+// h = <x_j, t'> and adds phi h to the warp's slot of the A_bar partial buffer
+// (read at the start of the path, so that its latency overlaps the first copy
+// group's, and written back at the end). The tiles differ in cost (their
+// paths' pair counts and degrees), so the host deals the CTAs of the single
+// wave to them in proportion to it; each warp of tile t serves every
+// (CTAs of t x warps)-th source.
 
 template <typename T>
 struct SrcSmem {
@@ -248,6 +253,18 @@ __device__ __forceinline__ void lds16(T* v, const T* src) {
   }
 }
 
+// Plain (coherent) load of CPL consecutive scalars that this kernel writes.
+template <int CPL, typename T>
+__device__ __forceinline__ void load_rw(T (&v)[CPL], const T* p) {
+  if constexpr (CPL == 2 && std::is_same<T, float>::value) {
+    const float2 t = *reinterpret_cast<const float2*>(p);
+    v[0] = t.x; v[1] = t.y;
+  } else {
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) v[c] = p[c];
+  }
+}
+
 template <typename T, int KP, int CPL, int G, int L1, int L2, int L3>
 __device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& pd, const SrcSmem<T>& s, int n,
                                          int slot, int chl, bool active, const T (&xs)[2 * L1 + 1][CPL],
@@ -255,16 +272,21 @@ __device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& 
   using CGp = cgt::CG<L1, L2, L3>;
   constexpr int D1 = 2 * L1 + 1, D3 = 2 * L3 + 1, NP = CGp::npair;
   constexpr int VW = sizeof(T) == 4 ? 4 : 2;
+  T* adst = p.apart + (size_t)slot * p.K * p.n_w + pd.w_off + chl;
   T a[KP][CPL], ab[KP][CPL];
 #pragma unroll
   for (int q = 0; q < KP; ++q) {
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) ab[q][c] = T(0);
     if (q < p.K) {
       load_ch<CPL>(a[q], p.A + (size_t)q * p.n_w + pd.w_off + chl);
+      if (active) {
+        load_rw<CPL>(ab[q], adst + (size_t)q * p.n_w);
+      } else {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) ab[q][c] = T(0);
+      }
     } else {
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) a[q][c] = T(0);
+      for (int c = 0; c < CPL; ++c) a[q][c] = ab[q][c] = T(0);
     }
   }
   // m_bar rows of the chunk's receivers go through a two-buffer ring of groups
@@ -354,27 +376,21 @@ __device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& 
   }
   }
   cp_wait<0>();
-  if (active && n > 0) {
+  if (active) {
 #pragma unroll
-    for (int q = 0; q < KP; ++q) {
-      if (q < p.K) {
-        T* dst = p.apart + ((size_t)slot * p.K + q) * p.n_w + pd.w_off + chl;
-        T v[CPL];
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) v[c] = dst[c] + ab[q][c];
-        store_ch<CPL>(dst, v);
-      }
-    }
+    for (int q = 0; q < KP; ++q)
+      if (q < p.K) store_ch<CPL>(adst + (size_t)q * p.n_w, ab[q]);
   }
 }
 
+// One warp's share of one input-block tile: sources slot, slot + stride, ...
 template <typename T, int KP, int CPL, class PR, int L1>
-__device__ __forceinline__ void src_tile(const UvuSrcParams<T>& p, const TileD& tl, int slot, int lane,
-                                         const SrcSmem<T>& s) {
+__device__ __forceinline__ void src_tile(const UvuSrcParams<T>& p, const TileD& tl, int slot, int stride,
+                                         int lane, const SrcSmem<T>& s) {
   constexpr int D1 = 2 * L1 + 1;
   const bool active = lane * CPL < tl.nch;
   const int chl = tl.ch0 + (active ? lane * CPL : 0);
-  for (int j = slot; j < p.N; j += p.n_slots) {
+  for (int j = slot; j < p.N; j += stride) {
     int k0 = ldg(p.colptr + j), k1 = ldg(p.colptr + j + 1);
     if (k0 < 0 || k1 < k0 || k1 > p.E) {
       raise_error(p.err, kErrCsr);
@@ -438,13 +454,16 @@ __global__ void __launch_bounds__(src_warps<T>() * 32, ctas_per_sm_for(sizeof(T)
 uvu_src_kernel(const __grid_constant__ UvuSrcParams<T> p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   // every warp of a CTA serves the same input-block tile (one family of path
-  // bodies per SM in the instruction cache); CTAs are tile-major
+  // bodies per SM in the instruction cache); the host deals the CTAs to the
+  // tiles in proportion to their per-edge cost
   constexpr int W = src_warps<T>();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int per_tile = (p.n_slots + W - 1) / W;
-  const int tile = blockIdx.x / per_tile;
-  const int slot = (blockIdx.x - tile * per_tile) * W + warp;
-  if (tile >= p.n_tiles || slot >= p.n_slots) return;
+  int tile = 0;
+  while (tile + 1 < p.n_tiles && (int)blockIdx.x >= p.tile_cta[tile + 1]) ++tile;
+  if (tile >= p.n_tiles || (int)blockIdx.x >= p.tile_cta[tile + 1]) return;
+  const int stride = min((p.tile_cta[tile + 1] - p.tile_cta[tile]) * W, p.n_slots);
+  const int slot = ((int)blockIdx.x - p.tile_cta[tile]) * W + warp;
+  if (slot >= stride) return;
   const TileD& tl = p.tiles[tile];
   unsigned char* base = smem_raw + (size_t)warp * p.warp_smem;
   SrcSmem<T> s;
@@ -452,7 +471,9 @@ uvu_src_kernel(const __grid_constant__ UvuSrcParams<T> p) {
   s.phi = reinterpret_cast<T*>(base + 32 * sizeof(int));
   s.cy = s.phi + 32 * KP;
   s.ring = reinterpret_cast<T*>(base + p.ring_off);
-  dispatch_l<PR::l1>(tl.l, [&](auto L) { src_tile<T, KP, CPL, PR, decltype(L)::value>(p, tl, slot, lane, s); });
+  dispatch_l<PR::l1>(tl.l, [&](auto L) {
+    src_tile<T, KP, CPL, PR, decltype(L)::value>(p, tl, slot, stride, lane, s);
+  });
 }
 
 template <typename T>
@@ -512,8 +533,7 @@ cudaError_t launch_uvu_src(const UvuSrcParams<T>& p, int prof, cudaStream_t s) {
   cudaError_t err = cudaMemsetAsync(p.apart, 0, sizeof(T) * (size_t)p.n_slots * p.K * p.n_w, s);
   if (err != cudaSuccess) return err;
   if (p.n_slots == 0 || p.n_tiles == 0 || p.N == 0) return cudaSuccess;
-  constexpr int W = src_warps<T>();
-  const unsigned blocks = (unsigned)(((long long)p.n_slots + W - 1) / W * p.n_tiles);
+  const unsigned blocks = (unsigned)p.tile_cta[p.n_tiles];
   switch (prof) {
     case 0: return launch_src_prof<T, KP, CPL, Prof<2, 2, 2>>(p, blocks, s);
     case 1: return launch_src_prof<T, KP, CPL, Prof<1, 3, 3>>(p, blocks, s);
