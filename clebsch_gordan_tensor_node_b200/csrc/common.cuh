@@ -59,6 +59,7 @@ struct UvuFwdParams {
   int chunk;                  // edges staged per warp at a time (<= 32)
   int warp_smem;              // bytes of shared memory per warp
   int ring_off;               // x copy ring: byte offset in the warp's slice
+  int split;                  // 1, or the warps of a CTA that share one task and deal its paths (small graphs)
   TileD tiles[kMaxTiles];     // one per (output block, channel tile)
   PathD paths[kMaxPaths];     // grouped by output block
 };
@@ -85,6 +86,7 @@ struct UvuSrcParams {         // backward: source-owned grad_x, grad_A partials
   int chunk;                  // edges staged per warp at a time (<= 32)
   int warp_smem;              // bytes of shared memory per warp
   int ring_off;               // m_bar copy ring: byte offset in the warp's slice
+  int split;                  // 1, or the warps of a CTA that share each source and deal the tile's paths
   int tile_cta[kMaxTiles + 1];  // CTAs [tile_cta[t], tile_cta[t + 1]) serve tile t
   TileD tiles[kMaxTiles];     // one per (input block, channel tile)
   PathD paths[kMaxPaths];     // grouped by input block

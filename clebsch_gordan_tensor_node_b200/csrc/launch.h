@@ -31,7 +31,7 @@ cudaError_t launch_uvu_edge_for(const Plan& P, const UvuEdgeParams<T>& p, cudaSt
 // on return it is the number the launch used (the tile partition's).
 template <typename T>
 cudaError_t launch_uvu_src_for(const Plan& P, UvuSrcParams<T>& p, cudaStream_t s) {
-  p.n_slots = uvu_src_partition(P, p.N, p.n_slots, p.tile_cta);
+  p.n_slots = uvu_src_partition(P, p.N, p.n_slots, p.tile_cta, &p.split);
   p.cy_stride = P.src_cy_stride;
   p.chunk = P.src_chunk;
   p.warp_smem = P.src_warp_smem;

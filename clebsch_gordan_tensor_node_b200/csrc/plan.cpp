@@ -350,6 +350,9 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
     P.src_ring_g = g;
     P.src_ring_off = base(chunk);
     P.src_warp_smem = per_warp(chunk);
+    // split mode adds the warps' x_bar partials (widest input block of the profile)
+    const int d1 = 2 * profs[P.prof][0] + 1;
+    P.src_split_ok = (size_t)per_warp(chunk) * warps + (size_t)warps * d1 * 32 * P.CPL * bsz <= 227 * 1024;
   }
   if (mode == TP_UVW) {
     if ((int)P.bout.size() > kMaxBlocks || (int)P.bin.size() > kMaxBlocks) {
@@ -476,16 +479,21 @@ int uvu_src_slots(const Plan& p, long long n_nodes) {
   return (int)s;
 }
 
-int uvu_src_partition(const Plan& p, long long n_nodes, long long max_slots, int* cta) {
+int uvu_src_partition(const Plan& p, long long n_nodes, long long max_slots, int* cta, int* split) {
   const int t = (int)p.in_tiles.size();
+  if (split) *split = 1;
   if (t == 0) {
     if (cta) cta[0] = 0;
     return 0;
   }
   const int bsz = p.dtype == TP_F32 ? 4 : 8;
-  const long long w = src_warps_for(bsz);
   const long long grid = std::max<long long>(t, (long long)kSMs * ctas_per_sm_for(bsz));
-  const long long cap = std::max<long long>(1, (n_nodes + w - 1) / w);   // CTAs with a source for every warp
+  // split mode while one warp per (source, tile) pair would not fill the
+  // wave's warps
+  const bool sp = p.src_split_ok && n_nodes * t <= grid * src_warps_for(bsz);
+  if (split && sp) *split = src_warps_for(bsz);
+  const long long w = sp ? 1 : src_warps_for(bsz);   // slots (source streams) per CTA
+  const long long cap = std::max<long long>(1, (n_nodes + w - 1) / w);   // CTAs with a source for every stream
   double tot = 0;
   for (int k = 0; k < t; ++k) tot += p.in_tile_cost[k];
   // proportional shares rounded down (at least one CTA each), then the CTAs
@@ -525,7 +533,7 @@ size_t workspace_bytes(const Plan& p, long long n_nodes, int pass) {
   size_t bytes = 0;
   if (p.mode == TP_UVU) {
     // first order: the source pass's slots; second order: its own source pass
-    if (pass == 1) bytes = (size_t)uvu_src_partition(p, n_nodes, 1LL << 40, nullptr) * p.K * p.n_w * b;
+    if (pass == 1) bytes = (size_t)uvu_src_partition(p, n_nodes, 1LL << 40, nullptr, nullptr) * p.K * p.n_w * b;
     if (pass >= 2) bytes = (size_t)uvu_src_slots(p, n_nodes) * p.K * p.n_w * b;
   } else {
     // packed A (forward operand; plus adjoint operand and packed A_bar in the

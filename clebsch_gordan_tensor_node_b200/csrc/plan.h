@@ -36,6 +36,7 @@ struct Plan {
   int fwd_ring_off = 0, fwd_ring_g = 1;   // forward: x copy ring offset (bytes); group size (= fwd_ring_g())
   int src_cy_stride = 0, src_chunk = 32, src_warp_smem = 0;
   int src_ring_off = 0, src_ring_g = 1;   // source pass: m_bar ring offset (bytes); group size (= src_ring_g())
+  bool src_split_ok = false;      // source pass: the split mode's x_bar partials fit beside the warps' slices
   std::vector<Block> bin, bout;
   std::vector<HostPath> paths;  // canonical enumeration order
   int c_in = 0, c_out = 0, dim_y = 0;
@@ -87,8 +88,11 @@ int uvu_src_slots(const Plan& p, long long n_nodes);
 // no more warps per tile than sources): tile t gets CTAs [cta[t], cta[t + 1])
 // when cta (n_tiles + 1 entries) is not null. Returns the A_bar partial slots,
 // the largest per-tile warp count capped at max_slots (each warp owns one slot
-// of its tile's columns and serves every slots-th source).
-int uvu_src_partition(const Plan& p, long long n_nodes, long long max_slots, int* cta);
+// of its tile's columns and serves every slots-th source). On graphs with too
+// few (source, tile) pairs to fill the GPU, *split (when not null) is set to
+// the warps of a CTA, which then share each source and deal the tile's paths;
+// a slot is then a CTA's. Otherwise *split = 1.
+int uvu_src_partition(const Plan& p, long long n_nodes, long long max_slots, int* cta, int* split = nullptr);
 
 // Bytes of workspace for pass 0 (forward) or 1 (backward) at n_nodes receivers.
 size_t workspace_bytes(const Plan& p, long long n_nodes, int pass);

@@ -222,7 +222,11 @@ uvu_edge_kernel(const __grid_constant__ UvuEdgeParams<T> p) {
 // group's, and written back at the end). The tiles differ in cost (their
 // paths' pair counts and degrees), so the host deals the CTAs of the single
 // wave to them in proportion to it; each warp of tile t serves every
-// (CTAs of t x warps)-th source.
+// (CTAs of t x warps)-th source. On graphs with too few (source, tile) pairs
+// to fill the GPU (split mode) the warps of a CTA share each source instead and
+// deal the tile's paths; their x_bar partials are added in warp order in shared
+// memory, and the CTA owns the slot (its warps write the columns of their own
+// paths).
 
 template <typename T>
 struct SrcSmem {
@@ -383,10 +387,11 @@ __device__ __forceinline__ void src_path(const UvuSrcParams<T>& p, const PathD& 
   }
 }
 
-// One warp's share of one input-block tile: sources slot, slot + stride, ...
+// One warp's share of one input-block tile: sources slot, slot + stride, ...,
+// and the paths pbeg + pw, pbeg + pw + ps, ... of each.
 template <typename T, int KP, int CPL, class PR, int L1>
 __device__ __forceinline__ void src_tile(const UvuSrcParams<T>& p, const TileD& tl, int slot, int stride,
-                                         int lane, const SrcSmem<T>& s) {
+                                         int lane, const SrcSmem<T>& s, int pw, int ps) {
   constexpr int D1 = 2 * L1 + 1;
   const bool active = lane * CPL < tl.nch;
   const int chl = tl.ch0 + (active ? lane * CPL : 0);
@@ -422,7 +427,7 @@ __device__ __forceinline__ void src_tile(const UvuSrcParams<T>& p, const TileD& 
         for (int q = 0; q < KP; ++q) s.phi[lane * KP + q] = ok ? ph[q] : T(0);
         const T* yrow = p.Y + (size_t)e * p.dim_y;
         T* cyrow = s.cy + lane * p.cy_stride;
-        for (int pi = tl.pbeg; pi < tl.pend; ++pi) {
+        for (int pi = tl.pbeg + pw; pi < tl.pend; pi += ps) {
           const PathD& pd = p.paths[pi];
           dispatch_l2l3<L1, PR::l2>(pd.l2, pd.l3, [&](auto A2, auto A3) {
             if constexpr (decltype(A3)::value <= PR::l3)
@@ -431,7 +436,7 @@ __device__ __forceinline__ void src_tile(const UvuSrcParams<T>& p, const TileD& 
         }
       }
       __syncwarp();
-      for (int pi = tl.pbeg; pi < tl.pend; ++pi) {
+      for (int pi = tl.pbeg + pw; pi < tl.pend; pi += ps) {
         const PathD& pd = p.paths[pi];
         dispatch_l2l3<L1, PR::l2>(pd.l2, pd.l3, [&](auto A2, auto A3) {
           if constexpr (decltype(A3)::value <= PR::l3)
@@ -440,6 +445,25 @@ __device__ __forceinline__ void src_tile(const UvuSrcParams<T>& p, const TileD& 
         });
       }
       __syncwarp();
+    }
+    if (ps > 1) {
+      // split mode: red[warp][m][32 CPL] after the warps' slices, added in warp order
+      extern __shared__ __align__(16) unsigned char smem_raw[];
+      constexpr int RW = 32 * CPL;
+      const int warp = threadIdx.x >> 5;
+      T* red = reinterpret_cast<T*>(smem_raw + (size_t)ps * p.warp_smem);
+      __syncthreads();   // the previous source's partials have been read
+#pragma unroll
+      for (int m = 0; m < D1; ++m)
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) red[(warp * D1 + m) * RW + lane * CPL + c] = gx[m][c];
+      __syncthreads();
+      if (warp != 0) continue;
+      for (int w = 1; w < ps; ++w)
+#pragma unroll
+        for (int m = 0; m < D1; ++m)
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) gx[m][c] += red[(w * D1 + m) * RW + lane * CPL + c];
     }
     if (active) {
       T* o = p.gx + (size_t)j * p.c_in + tl.off + chl;
@@ -461,9 +485,12 @@ uvu_src_kernel(const __grid_constant__ UvuSrcParams<T> p) {
   int tile = 0;
   while (tile + 1 < p.n_tiles && (int)blockIdx.x >= p.tile_cta[tile + 1]) ++tile;
   if (tile >= p.n_tiles || (int)blockIdx.x >= p.tile_cta[tile + 1]) return;
-  const int stride = min((p.tile_cta[tile + 1] - p.tile_cta[tile]) * W, p.n_slots);
-  const int slot = ((int)blockIdx.x - p.tile_cta[tile]) * W + warp;
-  if (slot >= stride) return;
+  // split mode: one source stream (slot) per CTA, whose warps deal the paths
+  const bool split = p.split > 1;
+  const int streams = split ? 1 : W;
+  const int stride = min((p.tile_cta[tile + 1] - p.tile_cta[tile]) * streams, p.n_slots);
+  const int slot = ((int)blockIdx.x - p.tile_cta[tile]) * streams + (split ? 0 : warp);
+  if (slot >= stride) return;   // uniform over the CTA in split mode
   const TileD& tl = p.tiles[tile];
   unsigned char* base = smem_raw + (size_t)warp * p.warp_smem;
   SrcSmem<T> s;
@@ -472,7 +499,7 @@ uvu_src_kernel(const __grid_constant__ UvuSrcParams<T> p) {
   s.cy = s.phi + 32 * KP;
   s.ring = reinterpret_cast<T*>(base + p.ring_off);
   dispatch_l<PR::l1>(tl.l, [&](auto L) {
-    src_tile<T, KP, CPL, PR, decltype(L)::value>(p, tl, slot, stride, lane, s);
+    src_tile<T, KP, CPL, PR, decltype(L)::value>(p, tl, slot, stride, lane, s, split ? warp : 0, split ? W : 1);
   });
 }
 
@@ -520,7 +547,9 @@ cudaError_t launch_uvu_edge(const UvuEdgeParams<T>& p0, int prof, cudaStream_t s
 
 template <typename T, int KP, int CPL, class PR>
 cudaError_t launch_src_prof(const UvuSrcParams<T>& p, unsigned blocks, cudaStream_t s) {
-  const size_t smem = (size_t)p.warp_smem * src_warps<T>();
+  constexpr int W = src_warps<T>();
+  const size_t smem = (size_t)p.warp_smem * W +
+                      (p.split > 1 ? sizeof(T) * (size_t)W * (2 * PR::l1 + 1) * 32 * CPL : 0);
   auto kern = uvu_src_kernel<T, KP, CPL, PR>;
   static SmemLimit limit;
   if (cudaError_t e = limit.ensure((const void*)kern, smem); e != cudaSuccess) return e;

@@ -25,6 +25,11 @@
 // Task order: windows of kWin receivers; inside a window all receivers of one
 // tile come first, so the warps of a CTA run the same code on neighbouring
 // receivers, and the window's x rows are re-read from L2 by the other tiles.
+//
+// Graphs with too few (receiver, tile) tasks to fill the GPU run in split mode:
+// a CTA takes one task and its warps deal the tile's paths round-robin, each
+// staging and sweeping the chunk for its own paths; their accumulators are
+// added in warp order in shared memory before the one store.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -187,7 +192,7 @@ __device__ __forceinline__ void fwd_path(const UvuFwdParams<T>& p, const PathD& 
 
 template <typename T, int KP, int CPL, int L1M, int L2M, int L3>
 __device__ __forceinline__ void fwd_tile(const UvuFwdParams<T>& p, const TileD& tl, int i, int lane,
-                                         const FwdSmem<T>& s) {
+                                         const FwdSmem<T>& s, int pw, int ps) {
   constexpr int D3 = 2 * L3 + 1;
   T acc[D3][CPL];
 #pragma unroll
@@ -219,7 +224,7 @@ __device__ __forceinline__ void fwd_tile(const UvuFwdParams<T>& p, const TileD& 
       for (int q = 0; q < KP; ++q) s.phi[lane * KP + q] = j < 0 ? T(0) : ph[q];
       const T* yrow = p.Y + (size_t)e * p.dim_y;
       T* cyrow = s.cy + lane * p.cy_stride;
-      for (int pi = tl.pbeg; pi < tl.pend; ++pi) {
+      for (int pi = tl.pbeg + pw; pi < tl.pend; pi += ps) {
         const PathD& pd = p.paths[pi];
         dispatch_l1l2<L3, L1M, L2M>(pd.l1, pd.l2, [&](auto A1, auto A2) {
           stage_cy<T, decltype(A1)::value, decltype(A2)::value, L3>(yrow, cyrow + pd.cy_off);
@@ -228,8 +233,8 @@ __device__ __forceinline__ void fwd_tile(const UvuFwdParams<T>& p, const TileD& 
       if (j < 0) s.j[lane] = 0;  // a skipped edge contributes zero (phi = 0)
     }
     __syncwarp();
-    // ---- sweep: every path of the tile over the staged chunk
-    for (int pi = tl.pbeg; pi < tl.pend; ++pi) {
+    // ---- sweep: every path of the tile (of this warp's share) over the staged chunk
+    for (int pi = tl.pbeg + pw; pi < tl.pend; pi += ps) {
       const PathD& pd = p.paths[pi];
       dispatch_l1l2<L3, L1M, L2M>(pd.l1, pd.l2, [&](auto A1, auto A2) {
         fwd_path<T, KP, CPL, fwd_ring_g(sizeof(T), CPL, L1M), decltype(A1)::value, decltype(A2)::value, L3>(
@@ -237,6 +242,26 @@ __device__ __forceinline__ void fwd_tile(const UvuFwdParams<T>& p, const TileD& 
       });
     }
     __syncwarp();
+  }
+  if (ps > 1) {
+    // split mode: red[warp][m][32 CPL] after the warps' slices, added in warp order
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    constexpr int RW = 32 * CPL;
+    const int warp = threadIdx.x >> 5;
+    T* red = reinterpret_cast<T*>(smem_raw + (size_t)ps * p.warp_smem);
+#pragma unroll
+    for (int m = 0; m < D3; ++m)
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) red[(warp * D3 + m) * RW + lane * CPL + c] = acc[m][c];
+    __syncthreads();
+    if (warp == 0) {
+      for (int w = 1; w < ps; ++w)
+#pragma unroll
+        for (int m = 0; m < D3; ++m)
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) acc[m][c] += red[(w * D3 + m) * RW + lane * CPL + c];
+    }
+    if (warp != 0) return;
   }
   if (active) {
     T* o = p.out + (size_t)i * p.c_out + tl.off + chl;
@@ -251,30 +276,38 @@ template <typename T, int KP, int CPL, int L1M, int L2M, int L3M>
 __global__ void __launch_bounds__(fwd_warps<T>() * 32, ctas_per_sm_for(sizeof(T)))
 uvu_fwd_kernel(const __grid_constant__ UvuFwdParams<T> p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const long long task = (long long)blockIdx.x * fwd_warps<T>() + warp;
+  const bool split = p.split > 1;   // split mode: one task per CTA, paths dealt to its warps
+  const long long task = split ? (long long)blockIdx.x : (long long)blockIdx.x * fwd_warps<T>() + warp;
   const long long per_win = (long long)kWin * p.n_tiles;
   const long long win = task / per_win;
   const int r = (int)(task - win * per_win);
   const int tile = r / kWin;
   const long long i = win * kWin + (r % kWin);
-  if (i >= p.N) return;
+  if (i >= p.N) return;   // uniform over the CTA in split mode
   const TileD& tl = p.tiles[tile];
   const FwdSmem<T> s = fwd_smem<T, KP>(p, warp);
   dispatch_l<L3M>(tl.l, [&](auto L) {
-    fwd_tile<T, KP, CPL, L1M, L2M, decltype(L)::value>(p, tl, (int)i, lane, s);
+    fwd_tile<T, KP, CPL, L1M, L2M, decltype(L)::value>(p, tl, (int)i, lane, s, split ? warp : 0,
+                                                       split ? p.split : 1);
   });
 }
 
 }  // namespace
 
 template <typename T, int KP, int CPL, int L1M, int L2M, int L3M>
-cudaError_t launch_uvu_fwd(const UvuFwdParams<T>& p, cudaStream_t s) {
+cudaError_t launch_uvu_fwd(const UvuFwdParams<T>& p0, cudaStream_t s) {
+  UvuFwdParams<T> p = p0;
   const long long wins = ((long long)p.N + kWin - 1) / kWin;
   const long long tasks = wins * kWin * p.n_tiles;
   if (tasks == 0) return cudaSuccess;
   constexpr int W = fwd_warps<T>();
-  const long long blocks = (tasks + W - 1) / W;
-  const size_t smem = (size_t)p.warp_smem * W;
+  // split mode while one warp per task would not fill the resident warp slots
+  // of one wave (and the warps' accumulators fit beside their slices)
+  const size_t red = sizeof(T) * (size_t)W * (2 * L3M + 1) * 32 * CPL;
+  const bool small = (long long)p.N * p.n_tiles <= (long long)kSMs * ctas_per_sm_for(sizeof(T)) * W;
+  p.split = small && (size_t)p.warp_smem * W + red <= (size_t)227 * 1024 ? W : 1;
+  const long long blocks = p.split > 1 ? tasks : (tasks + W - 1) / W;
+  const size_t smem = (size_t)p.warp_smem * W + (p.split > 1 ? red : 0);
   auto kern = uvu_fwd_kernel<T, KP, CPL, L1M, L2M, L3M>;
   static SmemLimit limit;
   if (cudaError_t e = limit.ensure((const void*)kern, smem); e != cudaSuccess) return e;
