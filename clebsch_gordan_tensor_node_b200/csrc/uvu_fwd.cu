@@ -120,8 +120,10 @@ __device__ __forceinline__ void fwd_path(const UvuFwdParams<T>& p, const PathD& 
     cp_commit();
     cp_wait<1>();   // this group's rows have landed
     const int tn = min(G, n - g0);
-#pragma unroll 1
-  for (int t = 0; t < tn; ++t) {
+    // the group's edges unrolled: their loads and FMA chains interleave
+#pragma unroll
+  for (int t = 0; t < G; ++t) {
+    if (t >= tn) break;
     const int k = g0 + t;
     T xv[D1][CPL];
     {
