@@ -292,9 +292,9 @@ def roofline_dbl(d, ms: float) -> dict:
 # summaries under profiles/ give the commands); absent where no capture of the
 # current kernels exists.
 NCU_TRAFFIC = {
-    (4, "fwdbwd"): (72_677_765_888, "uvu_fwd_kernel + uvu_edge_kernel + uvu_src_kernel + reduce_slots_kernel",
+    (4, "fwdbwd"): (73_558_277_120, "uvu_fwd_kernel + uvu_edge_kernel + uvu_src_kernel + reduce_slots_kernel",
                     "profiles/uvu_step_dram_large_100k.md"),
-    (4, "fwd"): (6_994_240_256 + 435_785_216, "uvu_fwd_kernel", "profiles/uvu_step_dram_large_100k.md"),
+    (4, "fwd"): (6_989_559_808 + 435_421_440, "uvu_fwd_kernel", "profiles/uvu_step_dram_large_100k.md"),
     (4, "dbl"): (112_633_031_680, "uvu_dbwd_recv_kernel + uvu_dbwd_edge_kernel + uvu_dbwd_src_kernel + "
                  "reduce_slots_kernel", "profiles/uvu_step_dram_large_100k.md"),
 }

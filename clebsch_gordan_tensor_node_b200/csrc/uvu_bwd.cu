@@ -121,8 +121,11 @@ __device__ __forceinline__ void edge_path(const UvuEdgeParams<T>& p, const PathD
   }
 }
 
+// fp32 up to degree 2: at most 128 registers, so that two CTAs (16 warps)
+// share an SM (a few spilled values); the wider profiles would spill kilobytes
+// under that cap and keep one CTA
 template <typename T, int KP, int V, class PR>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, sizeof(T) == 4 && PR::l3 <= 2 ? 2 : 1)
 uvu_edge_kernel(const __grid_constant__ UvuEdgeParams<T> p) {
   constexpr int DY = (PR::l2 + 1) * (PR::l2 + 1);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
