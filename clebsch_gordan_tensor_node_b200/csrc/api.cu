@@ -186,7 +186,7 @@ int double_backward_uvu(const Plan& P, const void* const* in, const int* const* 
     e = k8 ? launch_uvu_dbwd_edge<T, 8, 1>(p, P.prof, s) : launch_uvu_dbwd_edge<T, 16, 1>(p, P.prof, s);
   if (e != cudaSuccess) return cuda_fail(e, "double backward edge pass");
   // source pass: x_bar_dot and the A_bar_dot slot partials, then their sum
-  p.n_slots = uvu_src_slots(P, N);
+  p.n_slots = uvu_dbl_src_partition(P, N, p.tile_cta);
   copy_tables(p, P.dbl_in_tiles, P.dbl_paths_by_in);
   e = k8 ? launch_uvu_dbwd_src<T, 8, 1>(p, P.prof, s) : launch_uvu_dbwd_src<T, 16, 1>(p, P.prof, s);
   if (e != cudaSuccess) return cuda_fail(e, "double backward source pass");

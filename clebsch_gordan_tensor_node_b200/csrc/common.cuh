@@ -107,6 +107,7 @@ struct UvuDbwdParams {
   int N, E, K, c_in, c_out, dim_y, n_w;
   int n_paths, n_tiles, n_slots;
   int split;                  // edge pass: warps sharing one group of 32 edges
+  int tile_cta[kMaxTiles + 1];  // source pass: CTAs [tile_cta[t], tile_cta[t + 1]) serve tile t
   TileD tiles[kMaxTiles];     // receiver pass: (output block, 32-channel tile); source pass: input blocks
   PathD paths[kMaxPaths];     // receiver pass: by output block; source pass: by input block; edge pass: canonical
 };

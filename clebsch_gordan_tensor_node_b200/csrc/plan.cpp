@@ -329,6 +329,21 @@ int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_
     P.src_cy_stride = std::max(P.src_cy_stride, off);
     P.in_tile_cost.push_back(std::max(1, cost));
   }
+  // the second-order source pass's 32-channel tiles, by the same per-edge count
+  P.dbl_in_tile_cost.clear();
+  for (const TileD& t : P.dbl_in_tiles) {
+    int cost = 0;
+    for (int k = t.pbeg; k < t.pend; ++k) {
+      const PathD& d = P.dbl_paths_by_in[k];
+      auto e = real_cg_sparse(d.l1, d.l2, d.l3);
+      std::vector<std::pair<int, int>> pairs;
+      for (auto& q : e) pairs.emplace_back(q.m1, q.m3);
+      std::sort(pairs.begin(), pairs.end());
+      pairs.erase(std::unique(pairs.begin(), pairs.end()), pairs.end());
+      cost += (int)pairs.size() + 2 * (2 * d.l1 + 1) + 3 * P.K + (2 * d.l3 + 1);
+    }
+    P.dbl_in_tile_cost.push_back(std::max(1, cost));
+  }
   // source pass: per warp, the staged chunk (receivers, radial rows, cY) and an
   // m_bar copy ring of two groups of ring_g edges (every component of the
   // widest output block, 32 lanes x CPL channels). Group size, then chunk,
@@ -469,14 +484,52 @@ int uvw_chunk_rows(const Plan& p, long long n_nodes, int dir) {
   return (int)r;
 }
 
-int uvu_src_slots(const Plan& p, long long n_nodes) {
-  // one wave of source-pass CTAs, each serving one input-block tile
-  const long long t = std::max<long long>(1, (long long)p.in_tiles.size());
-  const int bsz = p.dtype == TP_F32 ? 4 : 8;
-  const int w = src_warps_for(bsz);
-  long long s = (long long)w * std::max<long long>(1, kSMs * ctas_per_sm_for(bsz) / t);
-  s = std::min<long long>(s, std::max<long long>(1, n_nodes));
-  return (int)s;
+// CTAs per tile in proportion to cost: shares rounded down (at least one CTA
+// each, at most cap), then the CTAs left over one at a time to the tile with the
+// most cost per CTA. Returns the largest count.
+long long deal_ctas(const std::vector<int>& cost, long long grid, long long cap, int* cta) {
+  const int t = (int)cost.size();
+  double tot = 0;
+  for (int k = 0; k < t; ++k) tot += cost[k];
+  std::vector<long long> c(t);
+  long long used = 0, most = 0;
+  for (int k = 0; k < t; ++k) {
+    c[k] = std::min(cap, std::max<long long>(1, (long long)(grid * (cost[k] / tot))));
+    used += c[k];
+  }
+  while (used < grid) {
+    int best = -1;
+    double bv = 0;
+    for (int k = 0; k < t; ++k) {
+      const double v = cost[k] / (double)c[k];
+      if (c[k] < cap && v > bv) {
+        bv = v;
+        best = k;
+      }
+    }
+    if (best < 0) break;
+    ++c[best];
+    ++used;
+  }
+  if (cta) cta[0] = 0;
+  for (int k = 0; k < t; ++k) {
+    most = std::max(most, c[k]);
+    if (cta) cta[k + 1] = cta[k] + (int)c[k];
+  }
+  return most;
+}
+
+int uvu_dbl_src_partition(const Plan& p, long long n_nodes, int* cta) {
+  const int t = (int)p.dbl_in_tiles.size();
+  if (t == 0) {
+    if (cta) cta[0] = 0;
+    return 0;
+  }
+  // several waves of CTAs (the hardware hands the later ones to the SMs that
+  // finish first), dealt to the tiles by cost
+  const long long grid = std::max<long long>(t, 4LL * kSMs);
+  const long long cap = std::max<long long>(1, (n_nodes + kDbWarps - 1) / kDbWarps);
+  return (int)(deal_ctas(p.dbl_in_tile_cost, grid, cap, cta) * kDbWarps);
 }
 
 int uvu_src_partition(const Plan& p, long long n_nodes, long long max_slots, int* cta, int* split) {
@@ -494,38 +547,8 @@ int uvu_src_partition(const Plan& p, long long n_nodes, long long max_slots, int
   if (split && sp) *split = src_warps_for(bsz);
   const long long w = sp ? 1 : src_warps_for(bsz);   // slots (source streams) per CTA
   const long long cap = std::max<long long>(1, (n_nodes + w - 1) / w);   // CTAs with a source for every stream
-  double tot = 0;
-  for (int k = 0; k < t; ++k) tot += p.in_tile_cost[k];
-  // proportional shares rounded down (at least one CTA each), then the CTAs
-  // left over one at a time to the tile with the most cost per CTA
-  std::vector<long long> c(t);
-  long long used = 0;
-  for (int k = 0; k < t; ++k) {
-    c[k] = std::min(cap, std::max<long long>(1, (long long)(grid * (p.in_tile_cost[k] / tot))));
-    used += c[k];
-  }
-  while (used < grid) {
-    int best = -1;
-    double bv = 0;
-    for (int k = 0; k < t; ++k) {
-      const double v = p.in_tile_cost[k] / (double)c[k];
-      if (c[k] < cap && v > bv) {
-        bv = v;
-        best = k;
-      }
-    }
-    if (best < 0) break;
-    ++c[best];
-    ++used;
-  }
-  long long slots = 0;
-  for (int k = 0; k < t; ++k) slots = std::max(slots, c[k] * w);
-  slots = std::max<long long>(1, std::min(slots, max_slots));
-  if (cta) {
-    cta[0] = 0;
-    for (int k = 0; k < t; ++k) cta[k + 1] = cta[k] + (int)c[k];
-  }
-  return (int)slots;
+  const long long slots = deal_ctas(p.in_tile_cost, grid, cap, cta) * w;
+  return (int)std::max<long long>(1, std::min(slots, max_slots));
 }
 
 size_t workspace_bytes(const Plan& p, long long n_nodes, int pass) {
@@ -534,7 +557,7 @@ size_t workspace_bytes(const Plan& p, long long n_nodes, int pass) {
   if (p.mode == TP_UVU) {
     // first order: the source pass's slots; second order: its own source pass
     if (pass == 1) bytes = (size_t)uvu_src_partition(p, n_nodes, 1LL << 40, nullptr, nullptr) * p.K * p.n_w * b;
-    if (pass >= 2) bytes = (size_t)uvu_src_slots(p, n_nodes) * p.K * p.n_w * b;
+    if (pass >= 2) bytes = (size_t)uvu_dbl_src_partition(p, n_nodes, nullptr) * p.K * p.n_w * b;
   } else {
     // packed A (forward operand; plus adjoint operand and packed A_bar in the
     // backward), each 256-byte aligned, and one (forward) or two (backward)

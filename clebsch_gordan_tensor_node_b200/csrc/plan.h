@@ -52,6 +52,7 @@ struct Plan {
   std::vector<TileD> dbl_out_tiles;
   std::vector<PathD> dbl_paths_by_out;
   std::vector<TileD> dbl_in_tiles;
+  std::vector<int> dbl_in_tile_cost;   // per-edge cost estimate of each dbl_in_tiles entry
   std::vector<PathD> dbl_paths_by_in;
   bool dbl_ok = false;
   // fully connected (uvw) tables
@@ -80,8 +81,11 @@ int uvw_chunk_rows(const Plan& p, long long n_nodes, int dir);
 int make_plan(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_radial, int mode,
               int dtype, Plan& out, std::string& msg, const int* sh_parity = nullptr);
 
-// Slots of the double-backward source pass's A_bar partial buffer (fixed per (plan, N)).
-int uvu_src_slots(const Plan& p, long long n_nodes);
+// CTAs of the double-backward source pass (kDbWarps warps each, one source
+// stream per warp), dealt to its 32-channel input tiles in proportion to their
+// per-edge cost as the first-order pass does; cta as in uvu_src_partition.
+// Returns the A_bar partial slots (the largest per-tile warp count).
+int uvu_dbl_src_partition(const Plan& p, long long n_nodes, int* cta);
 
 // CTAs of the first-order source pass, dealt to the input-block tiles in
 // proportion to their per-edge cost (one wave; at least one CTA per tile, and

@@ -22,6 +22,9 @@ constexpr int src_warps_for(int scalar_bytes) { return scalar_bytes == 4 ? 16 : 
 __host__ __device__
 #endif
 constexpr int ctas_per_sm_for(int scalar_bytes) { return scalar_bytes == 4 ? 1 : 2; }
+
+// Warps per CTA of the second-order passes (one channel per lane).
+constexpr int kDbWarps = 8;
 template <typename T>
 #ifdef __CUDACC__
 __host__ __device__

@@ -31,7 +31,6 @@
 namespace tpc {
 namespace {
 
-constexpr int kDbWarps = 8;
 constexpr long long kDbSplitGroups = 148LL * kDbWarps;   // 32-edge groups below which the edge pass splits
 
 template <int L1M, int L2M, int L3M>
@@ -377,11 +376,11 @@ __device__ __forceinline__ void src_path(const UvuDbwdParams<T>& p, const PathD&
 }
 
 template <typename T, int KP, class PR, int L1>
-__device__ __forceinline__ void src_tile(const UvuDbwdParams<T>& p, const TileD& tl, int slot, int lane) {
+__device__ __forceinline__ void src_tile(const UvuDbwdParams<T>& p, const TileD& tl, int slot, int stride, int lane) {
   constexpr int D1 = 2 * L1 + 1;
   const bool active = lane < tl.nch;
   const int ch = tl.ch0 + (active ? lane : 0);
-  for (int j = slot; j < p.N; j += p.n_slots) {
+  for (int j = slot; j < p.N; j += stride) {
     int k0 = ldg(p.colptr + j), k1 = ldg(p.colptr + j + 1);
     if (k0 < 0 || k1 < k0 || k1 > p.E) {
       raise_error(p.err, kErrCsr);
@@ -415,12 +414,15 @@ __device__ __forceinline__ void src_tile(const UvuDbwdParams<T>& p, const TileD&
 template <typename T, int KP, class PR>
 __global__ void __launch_bounds__(kDbWarps * 32) uvu_dbwd_src_kernel(const __grid_constant__ UvuDbwdParams<T> p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int per_tile = (p.n_slots + kDbWarps - 1) / kDbWarps;
-  const int tile = blockIdx.x / per_tile;
-  const int slot = (blockIdx.x - tile * per_tile) * kDbWarps + warp;
-  if (tile >= p.n_tiles || slot >= p.n_slots) return;
+  // the host deals the CTAs to the tiles in proportion to their per-edge cost
+  int tile = 0;
+  while (tile + 1 < p.n_tiles && (int)blockIdx.x >= p.tile_cta[tile + 1]) ++tile;
+  if (tile >= p.n_tiles || (int)blockIdx.x >= p.tile_cta[tile + 1]) return;
+  const int stride = min((p.tile_cta[tile + 1] - p.tile_cta[tile]) * kDbWarps, p.n_slots);
+  const int slot = ((int)blockIdx.x - p.tile_cta[tile]) * kDbWarps + warp;
+  if (slot >= stride) return;
   const TileD& tl = p.tiles[tile];
-  dispatch_l<PR::l1>(tl.l, [&](auto L) { src_tile<T, KP, PR, decltype(L)::value>(p, tl, slot, lane); });
+  dispatch_l<PR::l1>(tl.l, [&](auto L) { src_tile<T, KP, PR, decltype(L)::value>(p, tl, slot, stride, lane); });
 }
 
 // Wide: the degree-6 profile is compiled (fp32, K <= 8, scalar gathers only).
@@ -479,7 +481,7 @@ cudaError_t launch_uvu_dbwd_src(const UvuDbwdParams<T>& p, int prof, cudaStream_
   cudaError_t err = cudaMemsetAsync(p.apart, 0, sizeof(T) * (size_t)p.n_slots * p.K * p.n_w, s);
   if (err != cudaSuccess) return err;
   if (p.n_slots == 0 || p.n_tiles == 0 || p.N == 0) return cudaSuccess;
-  const unsigned blocks = (unsigned)(((long long)p.n_slots + kDbWarps - 1) / kDbWarps * p.n_tiles);
+  const unsigned blocks = (unsigned)p.tile_cta[p.n_tiles];
   return by_prof<wide_ok<T, KP>()>(prof, [&](auto PR) {
     uvu_dbwd_src_kernel<T, KP, decltype(PR)><<<blocks, kDbWarps * 32, 0, s>>>(p);
     return cudaGetLastError();
