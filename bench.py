@@ -295,7 +295,7 @@ NCU_TRAFFIC = {
     (4, "fwdbwd"): (73_558_277_120, "uvu_fwd_kernel + uvu_edge_kernel + uvu_src_kernel + reduce_slots_kernel",
                     "profiles/uvu_step_dram_large_100k.md"),
     (4, "fwd"): (6_989_559_808 + 435_421_440, "uvu_fwd_kernel", "profiles/uvu_step_dram_large_100k.md"),
-    (4, "dbl"): (112_633_031_680, "uvu_dbwd_recv_kernel + uvu_dbwd_edge_kernel + uvu_dbwd_src_kernel + "
+    (4, "dbl"): (107_987_648_000, "uvu_dbwd_recv_kernel + uvu_dbwd_edge_kernel + uvu_dbwd_src_kernel + "
                  "reduce_slots_kernel", "profiles/uvu_step_dram_large_100k.md"),
 }
 
